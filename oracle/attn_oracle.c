@@ -1,0 +1,403 @@
+/*
+ * attn_oracle.c -- plain fp64 CPU oracle for exact scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker the CUDA library is compared
+ * against.  Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * load it; the product path (the CUDA library and its Python binding) never does, and
+ * the two share no code, headers, tables or helpers.
+ *
+ * What it computes is the plain definition of attention, written out row by row in
+ * double precision, with no tiling, no online softmax and no reordering:
+ *
+ *   Step 1  S = scale * Q K^T, with S_ij = -inf where the causal mask hides key j > i.
+ *   Step 2  P = softmax(S) per row: m_i = max_j S_ij, l_i = sum_j exp(S_ij - m_i),
+ *           P_ij = exp(S_ij - m_i) / l_i; the saved statistic is LSE_i = m_i + ln l_i.
+ *   Step 3  O = P V.
+ *
+ * Sources: "FlashAttention 与高效注意力内核：IO 感知与分块计算" (plumephp.com tutorial),
+ * section "标准注意力三步" (S = Q K^T, P = softmax(S), O = P V) and section "前向" (only O
+ * and the softmax statistics m, l are kept); "Flash-Attention" concept page
+ * (awesome-system-papers), section "核心思想" (the 1/sqrt(d) scale inside the softmax).
+ *
+ * Backward: the standard analytic chain rule through the softmax, with the gradient of
+ * the scaled scores S = scale * Q K^T:
+ *   D_i   = sum_c dO_ic O_ic
+ *   dP_ij = dO_i . V_j
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij K_j
+ *   dK_j  = scale * sum_i dS_ij Q_i      (summed over the query heads that share K_j)
+ *   dV_j  = sum_i P_ij dO_i              (summed likewise)
+ * The tutorial's section "反向" says only that the backward recomputes S and P from
+ * Q/K/V and the saved statistics and then forms dQ/dK/dV from dO; the formulas above are
+ * the plain derivative of the forward definition.  Here P_ij is re-formed from the saved
+ * LSE as exp(S_ij - LSE_i), which equals exp(S_ij - m_i) / l_i by definition.
+ *
+ * Grouped-query attention ("相关工作" page, paper 6 "Grouped-Query Attention"): query
+ * head h reads key/value head floor(h * hkv / hq), i.e. contiguous groups of hq/hkv
+ * query heads share one K/V head.  Variable-length packing ("验证清单": 变长序列打包):
+ * sequences are concatenated along the token axis, described by cu_seqlens (prefix sums,
+ * cu_seqlens[0] = 0), and attention never crosses a sequence boundary.
+ *
+ * Layouts (all row-major, double):  q, o, dout, dq : [T, hq, d]
+ *                                   k, v, dk, dv   : [T, hkv, d]
+ *                                   lse            : [hq, T]
+ * A query row with no visible key (impossible for causal self-attention with length >= 1)
+ * gets O = 0 and LSE = -inf.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEM 2
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    const int32_t *cu;
+    int32_t nseq, hq, hkv, d, causal;
+    double scale;
+    const uint8_t *row_sel;  /* optional: only rows with row_sel[t] != 0 are produced */
+    const uint8_t *key_sel;  /* optional: only keys with key_sel[t] != 0 get dK/dV */
+    double *o, *lse, *dd;    /* forward results (and D for the backward) */
+    double *dq, *dk, *dv;
+} problem;
+
+/* ---- the three steps, for one query row -------------------------------------------- */
+
+/* Number of keys row i (0-based inside its sequence of length n) may look at. */
+static int visible_keys(int i, int n, int causal) { return causal ? i + 1 : n; }
+
+/* Step 1: s_j = scale * <q_i, k_j> for visible keys, -inf for hidden ones. */
+static void score_row(const problem *P, int64_t row, int64_t key0, int n, int vis, int h, double *s)
+{
+    const int d = P->d;
+    const int g = (int)(((int64_t)h * P->hkv) / P->hq);
+    const double *qi = P->q + (row * P->hq + h) * d;
+    for (int j = 0; j < n; ++j) {
+        if (j >= vis) { s[j] = -INFINITY; continue; }
+        const double *kj = P->k + ((key0 + j) * P->hkv + g) * d;
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qi[c] * kj[c];
+        s[j] = P->scale * acc;
+    }
+}
+
+/* Step 2: p_j = exp(s_j - m) / l with m = max s, l = sum exp(s_j - m); returns LSE = m + ln l. */
+static double softmax_row(const double *s, int n, double *p)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) if (s[j] > m) m = s[j];
+    if (m == -INFINITY) { for (int j = 0; j < n; ++j) p[j] = 0.0; return -INFINITY; }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) { p[j] = exp(s[j] - m); l += p[j]; }
+    for (int j = 0; j < n; ++j) p[j] /= l;
+    return m + log(l);
+}
+
+/* Step 3: o_i = sum_j p_j v_j. */
+static void output_row(const problem *P, int64_t key0, int n, int h, const double *p, double *oi)
+{
+    const int d = P->d;
+    const int g = (int)(((int64_t)h * P->hkv) / P->hq);
+    for (int c = 0; c < d; ++c) oi[c] = 0.0;
+    for (int j = 0; j < n; ++j) {
+        if (p[j] == 0.0) continue;
+        const double *vj = P->v + ((key0 + j) * P->hkv + g) * d;
+        for (int c = 0; c < d; ++c) oi[c] += p[j] * vj[c];
+    }
+}
+
+/* ---- work items and threads -------------------------------------------------------- */
+
+#define ROWS_PER_ITEM 32
+
+typedef struct {
+    problem *P;
+    int kind;            /* 0: forward rows, 1: dQ rows, 2: dK/dV keys */
+    int64_t nitems;
+    int64_t *item_seq;   /* item -> sequence */
+    int64_t *item_head;  /* item -> head (query head for kinds 0/1, kv head for kind 2) */
+    int64_t *item_row0;  /* item -> first row (inside the sequence) */
+    int64_t next;
+    pthread_mutex_t lock;
+    int failed;
+} workset;
+
+static void do_forward_rows(problem *P, int64_t seq, int h, int r0, int r1, double *s, double *p)
+{
+    const int64_t t0 = P->cu[seq];
+    const int n = (int)(P->cu[seq + 1] - t0);
+    for (int i = r0; i < r1; ++i) {
+        const int64_t row = t0 + i;
+        if (P->row_sel && !P->row_sel[row]) continue;
+        const int vis = visible_keys(i, n, P->causal);
+        score_row(P, row, t0, n, vis, h, s);
+        const double lse = softmax_row(s, n, p);
+        double *oi = P->o + (row * P->hq + h) * P->d;
+        output_row(P, t0, n, h, p, oi);
+        P->lse[(int64_t)h * P->cu[P->nseq] + row] = lse;
+        if (P->dd) {  /* D_i = sum_c dO_ic O_ic, needed by the backward */
+            const double *doi = P->dout + (row * P->hq + h) * P->d;
+            double acc = 0.0;
+            for (int c = 0; c < P->d; ++c) acc += doi[c] * oi[c];
+            P->dd[(int64_t)h * P->cu[P->nseq] + row] = acc;
+        }
+    }
+}
+
+/* dS_ij for keys j in [j0, j1) of one row (all visible), given the saved LSE_i and D_i:
+ * P_ij = exp(S_ij - LSE_i), dS_ij = P_ij (dP_ij - D_i).  p[j] and ds[j] are written for
+ * j in [j0, j1) only. */
+static void ds_row(const problem *P, int64_t row, int64_t key0, int j0, int j1, int h,
+                   double *ds, double *p)
+{
+    const int d = P->d;
+    const int g = (int)(((int64_t)h * P->hkv) / P->hq);
+    const int64_t T = P->cu[P->nseq];
+    const double lse = P->lse[(int64_t)h * T + row];
+    const double Di = P->dd[(int64_t)h * T + row];
+    const double *qi = P->q + (row * P->hq + h) * d;
+    const double *doi = P->dout + (row * P->hq + h) * d;
+    for (int j = j0; j < j1; ++j) {
+        const double *kj = P->k + ((key0 + j) * P->hkv + g) * d;
+        const double *vj = P->v + ((key0 + j) * P->hkv + g) * d;
+        double sc = 0.0, dp = 0.0;
+        for (int c = 0; c < d; ++c) { sc += qi[c] * kj[c]; dp += doi[c] * vj[c]; }
+        p[j] = exp(P->scale * sc - lse);
+        ds[j] = p[j] * (dp - Di);
+    }
+}
+
+static void do_dq_rows(problem *P, int64_t seq, int h, int r0, int r1, double *s, double *p)
+{
+    const int64_t t0 = P->cu[seq];
+    const int n = (int)(P->cu[seq + 1] - t0);
+    const int d = P->d;
+    const int g = (int)(((int64_t)h * P->hkv) / P->hq);
+    for (int i = r0; i < r1; ++i) {
+        const int64_t row = t0 + i;
+        if (P->row_sel && !P->row_sel[row]) continue;
+        const int vis = visible_keys(i, n, P->causal);
+        ds_row(P, row, t0, 0, vis, h, s, p);
+        double *dqi = P->dq + (row * P->hq + h) * d;
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+        for (int j = 0; j < vis; ++j) {
+            const double *kj = P->k + ((t0 + j) * P->hkv + g) * d;
+            for (int c = 0; c < d; ++c) dqi[c] += s[j] * kj[c];
+        }
+        for (int c = 0; c < d; ++c) dqi[c] *= P->scale;
+    }
+}
+
+/* dK_j, dV_j for keys j in [r0, r1) of one kv head: sum over the query heads of its
+ * group and over every query row that sees key j. */
+static void do_dkdv_keys(problem *P, int64_t seq, int g, int r0, int r1, double *s, double *p)
+{
+    const int64_t t0 = P->cu[seq];
+    const int n = (int)(P->cu[seq + 1] - t0);
+    const int d = P->d;
+    const int G = P->hq / P->hkv;
+    double *acck = (double *)calloc((size_t)(r1 - r0) * d, sizeof(double));
+    double *accv = (double *)calloc((size_t)(r1 - r0) * d, sizeof(double));
+    if (!acck || !accv) { free(acck); free(accv); return; }
+    int any = 0;
+    for (int j = r0; j < r1; ++j) if (!P->key_sel || P->key_sel[t0 + j]) any = 1;
+    if (any) {
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            for (int i = 0; i < n; ++i) {
+                const int vis = visible_keys(i, n, P->causal);
+                if (vis <= r0) continue;  /* row i sees none of these keys */
+                const int64_t row = t0 + i;
+                const int j1 = r1 < vis ? r1 : vis;
+                ds_row(P, row, t0, r0, j1, h, s, p);
+                const double *qi = P->q + (row * P->hq + h) * d;
+                const double *doi = P->dout + (row * P->hq + h) * d;
+                for (int j = r0; j < j1; ++j) {
+                    double *ak = acck + (size_t)(j - r0) * d;
+                    double *av = accv + (size_t)(j - r0) * d;
+                    for (int c = 0; c < d; ++c) { ak[c] += s[j] * qi[c]; av[c] += p[j] * doi[c]; }
+                }
+            }
+        }
+    }
+    for (int j = r0; j < r1; ++j) {
+        const int64_t key = t0 + j;
+        if (P->key_sel && !P->key_sel[key]) continue;
+        double *dkj = P->dk + (key * P->hkv + g) * d;
+        double *dvj = P->dv + (key * P->hkv + g) * d;
+        for (int c = 0; c < d; ++c) {
+            dkj[c] = P->scale * acck[(size_t)(j - r0) * d + c];
+            dvj[c] = accv[(size_t)(j - r0) * d + c];
+        }
+    }
+    free(acck);
+    free(accv);
+}
+
+static void *worker(void *arg)
+{
+    workset *W = (workset *)arg;
+    problem *P = W->P;
+    int64_t maxn = 0;
+    for (int b = 0; b < P->nseq; ++b) {
+        const int64_t n = P->cu[b + 1] - P->cu[b];
+        if (n > maxn) maxn = n;
+    }
+    double *s = (double *)malloc((size_t)(maxn > 0 ? maxn : 1) * sizeof(double));
+    double *p = (double *)malloc((size_t)(maxn > 0 ? maxn : 1) * sizeof(double));
+    if (!s || !p) {
+        pthread_mutex_lock(&W->lock); W->failed = 1; pthread_mutex_unlock(&W->lock);
+        free(s); free(p);
+        return NULL;
+    }
+    for (;;) {
+        pthread_mutex_lock(&W->lock);
+        const int64_t it = W->next++;
+        pthread_mutex_unlock(&W->lock);
+        if (it >= W->nitems) break;
+        const int64_t seq = W->item_seq[it];
+        const int h = (int)W->item_head[it];
+        const int r0 = (int)W->item_row0[it];
+        const int n = (int)(P->cu[seq + 1] - P->cu[seq]);
+        const int r1 = r0 + ROWS_PER_ITEM < n ? r0 + ROWS_PER_ITEM : n;
+        if (W->kind == 0) do_forward_rows(P, seq, h, r0, r1, s, p);
+        else if (W->kind == 1) do_dq_rows(P, seq, h, r0, r1, s, p);
+        else do_dkdv_keys(P, seq, h, r0, r1, s, p);
+    }
+    free(s);
+    free(p);
+    return NULL;
+}
+
+static int run_items(problem *P, int kind, int nheads, int nthreads)
+{
+    int64_t nitems = 0;
+    for (int b = 0; b < P->nseq; ++b) {
+        const int64_t n = P->cu[b + 1] - P->cu[b];
+        nitems += (int64_t)nheads * ((n + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM);
+    }
+    workset W;
+    memset(&W, 0, sizeof W);
+    W.P = P;
+    W.kind = kind;
+    W.nitems = nitems;
+    W.item_seq = (int64_t *)malloc((size_t)(nitems > 0 ? nitems : 1) * sizeof(int64_t));
+    W.item_head = (int64_t *)malloc((size_t)(nitems > 0 ? nitems : 1) * sizeof(int64_t));
+    W.item_row0 = (int64_t *)malloc((size_t)(nitems > 0 ? nitems : 1) * sizeof(int64_t));
+    if (!W.item_seq || !W.item_head || !W.item_row0) {
+        free(W.item_seq); free(W.item_head); free(W.item_row0);
+        return ORACLE_NO_MEM;
+    }
+    int64_t it = 0;
+    for (int b = 0; b < P->nseq; ++b) {
+        const int64_t n = P->cu[b + 1] - P->cu[b];
+        for (int h = 0; h < nheads; ++h)
+            for (int64_t r = 0; r < n; r += ROWS_PER_ITEM) {
+                W.item_seq[it] = b; W.item_head[it] = h; W.item_row0[it] = r; ++it;
+            }
+    }
+    pthread_mutex_init(&W.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    pthread_t *tid = (pthread_t *)malloc((size_t)nthreads * sizeof(pthread_t));
+    int started = 0;
+    if (tid) {
+        for (; started < nthreads; ++started)
+            if (pthread_create(&tid[started], NULL, worker, &W) != 0) break;
+    }
+    if (started == 0) worker(&W);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    free(tid);
+    pthread_mutex_destroy(&W.lock);
+    free(W.item_seq); free(W.item_head); free(W.item_row0);
+    return W.failed ? ORACLE_NO_MEM : ORACLE_OK;
+}
+
+static int check_args(const int32_t *cu, int32_t nseq, int32_t hq, int32_t hkv, int32_t d)
+{
+    if (!cu || nseq < 0 || hq <= 0 || hkv <= 0 || d <= 0 || hq % hkv != 0) return ORACLE_BAD_ARG;
+    if (cu[0] != 0) return ORACLE_BAD_ARG;
+    for (int b = 0; b < nseq; ++b) if (cu[b + 1] < cu[b]) return ORACLE_BAD_ARG;
+    return ORACLE_OK;
+}
+
+/* Forward: o [T,hq,d], lse [hq,T].  row_sel (optional, [T]) restricts which rows are
+ * written; other entries of o and lse are left untouched. */
+int oracle_attn_fwd(const double *q, const double *k, const double *v,
+                    const int32_t *cu_seqlens, int32_t nseq,
+                    int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                    const uint8_t *row_sel, double *o, double *lse, int32_t nthreads)
+{
+    int rc = check_args(cu_seqlens, nseq, hq, hkv, d);
+    if (rc) return rc;
+    problem P;
+    memset(&P, 0, sizeof P);
+    P.q = q; P.k = k; P.v = v; P.cu = cu_seqlens; P.nseq = nseq;
+    P.hq = hq; P.hkv = hkv; P.d = d; P.scale = scale; P.causal = causal;
+    P.row_sel = row_sel; P.o = o; P.lse = lse;
+    return run_items(&P, 0, hq, nthreads);
+}
+
+/* Backward: dq [T,hq,d], dk/dv [T,hkv,d].  The oracle forms its own O, LSE and D from
+ * the definition first (all rows of every head).  row_sel / key_sel (optional, [T])
+ * restrict which dQ rows and which dK/dV keys are produced; others stay untouched.
+ * o_out / lse_out (optional) receive the forward results. */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    const int32_t *cu_seqlens, int32_t nseq,
+                    int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                    const uint8_t *row_sel, const uint8_t *key_sel,
+                    double *dq, double *dk, double *dv,
+                    double *o_out, double *lse_out, int32_t nthreads)
+{
+    int rc = check_args(cu_seqlens, nseq, hq, hkv, d);
+    if (rc) return rc;
+    const int64_t T = cu_seqlens[nseq];
+    double *o = o_out ? o_out : (double *)malloc((size_t)(T > 0 ? T : 1) * hq * d * sizeof(double));
+    double *lse = lse_out ? lse_out : (double *)malloc((size_t)(T > 0 ? T : 1) * hq * sizeof(double));
+    double *dd = (double *)malloc((size_t)(T > 0 ? T : 1) * hq * sizeof(double));
+    if (!o || !lse || !dd) {
+        if (!o_out) free(o);
+        if (!lse_out) free(lse);
+        free(dd);
+        return ORACLE_NO_MEM;
+    }
+    problem P;
+    memset(&P, 0, sizeof P);
+    P.q = q; P.k = k; P.v = v; P.dout = dout; P.cu = cu_seqlens; P.nseq = nseq;
+    P.hq = hq; P.hkv = hkv; P.d = d; P.scale = scale; P.causal = causal;
+    P.o = o; P.lse = lse; P.dd = dd;
+    P.dq = dq; P.dk = dk; P.dv = dv;
+    rc = run_items(&P, 0, hq, nthreads);          /* O, LSE, D for every row */
+    if (!rc) { P.row_sel = row_sel; rc = run_items(&P, 1, hq, nthreads); }   /* dQ rows */
+    if (!rc) { P.row_sel = NULL; P.key_sel = key_sel; rc = run_items(&P, 2, hkv, nthreads); } /* dK, dV */
+    if (!o_out) free(o);
+    if (!lse_out) free(lse);
+    free(dd);
+    return rc;
+}
+
+/* The probability matrix of one (sequence, head) problem, materialised: p [n, n].
+ * q [n,d], k [n,d].  Used by the tests for the row-sum / mask invariants. */
+int oracle_attn_probs(const double *q, const double *k, int32_t n, int32_t d,
+                      double scale, int32_t causal, double *p, double *lse)
+{
+    if (n < 0 || d <= 0) return ORACLE_BAD_ARG;
+    int32_t cu[2] = {0, n};
+    problem P;
+    memset(&P, 0, sizeof P);
+    P.q = q; P.k = k; P.cu = cu; P.nseq = 1; P.hq = 1; P.hkv = 1; P.d = d;
+    P.scale = scale; P.causal = causal;
+    double *s = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    if (!s) return ORACLE_NO_MEM;
+    for (int i = 0; i < n; ++i) {
+        score_row(&P, i, 0, n, visible_keys(i, n, causal), 0, s);
+        const double l = softmax_row(s, n, p + (size_t)i * n);
+        if (lse) lse[i] = l;
+    }
+    free(s);
+    return ORACLE_OK;
+}

@@ -1,0 +1,71 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of ``oracle/attn_oracle.c`` (a dropped term, a
+wrong sign, a wrong index or a transposed operand), builds it on the CPU, and runs the
+battery of pins from ``test_oracle`` against it.  Every mutant must fail at least one.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
+
+MUTANTS = {
+    "scale dropped from the scores": ("s[j] = P->scale * acc;", "s[j] = acc;"),
+    "causal mask off by one": ("return causal ? i + 1 : n;", "return causal ? i + 2 : n;"),
+    "GQA head mapping interleaved": ("const int g = (int)(((int64_t)h * P->hkv) / P->hq);\n    const double *qi = P->q + (row",
+                                     "const int g = h % P->hkv;\n    const double *qi = P->q + (row"),
+    "max dropped from LSE": ("return m + log(l);", "return log(l);"),
+    "softmax not normalised": ("p[j] /= l;", "p[j] /= 1.0;"),
+    "wrong sign in dS": ("ds[j] = p[j] * (dp - Di);", "ds[j] = p[j] * (dp + Di);"),
+    "D from the wrong vector": ("acc += doi[c] * oi[c];", "acc += doi[c] * doi[c];"),
+    "dK missing the scale": ("dkj[c] = P->scale * acck", "dkj[c] = acck"),
+    "dV with Q in place of dO": ("av[c] += p[j] * doi[c];", "av[c] += p[j] * qi[c];"),
+    "dQ with V in place of K": ("const double *kj = P->k + ((t0 + j) * P->hkv + g) * d;\n            for (int c = 0; c < d; ++c) dqi[c]",
+                                "const double *kj = P->v + ((t0 + j) * P->hkv + g) * d;\n            for (int c = 0; c < d; ++c) dqi[c]"),
+    "score mask boundary off by one": ("if (j >= vis) { s[j] = -INFINITY; continue; }", "if (j > vis) { s[j] = -INFINITY; continue; }"),
+    "value row from the wrong key": ("const double *vj = P->v + ((key0 + j) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]",
+                                     "const double *vj = P->v + ((key0 + (n - 1 - j)) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]"),
+}
+
+
+def _battery():
+    """True when every pin passes."""
+    checks = [
+        lambda: pins.test_forward_matches_brute_force([3, 7, 1], 4, 2, 2, True),
+        lambda: pins.test_forward_matches_brute_force([8], 2, 2, 4, False),
+        lambda: pins.test_matches_torch_sdpa_and_autograd(20, 6, 3, 5, True),
+        lambda: pins.test_matches_torch_sdpa_and_autograd(9, 2, 2, 8, False),
+        lambda: pins.test_gradients_match_finite_differences(True),
+        lambda: pins.test_worked_example_online_merge(),
+        lambda: pins.test_zero_queries_give_uniform_average(True),
+        lambda: pins.test_gradient_invariants(False),
+    ]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def test_unmutated_oracle_passes_battery():
+    assert _battery()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                           "-o", str(lib), str(mutated), "-lm"])
+    with oracle.using_library(str(lib)):
+        assert not _battery(), f"mutant {name!r} passed every pin"
