@@ -1,0 +1,129 @@
+/*
+ * attn.h -- C ABI of libattn.so: exact scaled-dot-product attention, forward and
+ * backward, on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (the "FlashAttention 与高效注意力内核：IO 感知与分块计算" tutorial,
+ * section 标准注意力三步, with the 1/sqrt(d)-style scale of the "Flash-Attention" concept
+ * page, section 核心思想):
+ *
+ *     S = scale * Q K^T   (S_ij = -inf where causal and key j > query i)
+ *     P = softmax(S)      row by row
+ *     O = P V
+ *
+ * computed IO-aware: Q/K/V tiles are staged in on-chip memory, the softmax is the
+ * online (running max m, running sum l, rescaled running O) form of the tutorial's
+ * section "Online Softmax 技巧", and only O and the per-row statistic
+ * LSE_i = m_i + ln l_i (natural log, in units of the scaled scores) reach HBM (section
+ * "前向").  The backward recomputes S and P from Q, K, V and LSE (section "反向") and
+ * applies D_i = sum_c dO_ic O_ic, dP = dO V^T, dS = P o (dP - D),
+ * dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+ *
+ * Grouped-query attention ("相关工作" page, paper 6): query head h reads K/V head
+ * h / (hq / hkv).  Variable-length packing (the tutorial's 验证清单, 变长序列打包):
+ * sequences are concatenated on the token axis and described by cu_seqlens; attention
+ * never crosses a sequence boundary; a zero-length sequence is legal and writes nothing.
+ * Causal masking is top-left aligned inside each sequence: query i sees keys j <= i.
+ *
+ * ---- Conventions shared by every entry point ----------------------------------------
+ *
+ * Layouts (row-major, innermost dimension contiguous, no padding):
+ *     q, o, dout, dq   [total_tokens, hq,  d]
+ *     k, v, dk, dv     [total_tokens, hkv, d]
+ *     lse              [hq, total_tokens]            float32
+ * Element type: ATTN_BF16 -- q/k/v/o/dout/dq/dk/dv are bfloat16, statistics and all
+ * accumulation are float32; ATTN_FP32 -- the fp32-input check mode, every tensor is
+ * float32 (computed with float32 arithmetic throughout; slow, for numerical checks).
+ *
+ * Shapes: batch mode passes cu_seqlens = NULL, `batch` sequences of `seqlen` tokens,
+ * total_tokens = batch * seqlen.  Varlen mode passes cu_seqlens, a DEVICE int32 array of
+ * batch + 1 prefix sums with cu_seqlens[0] = 0 and cu_seqlens[batch] = total_tokens;
+ * `seqlen` is ignored and `max_seqlen` must be >= every sequence length (a sequence
+ * longer than max_seqlen is reported by attn_get_device_error as ATTN_ERR_INVALID_ARG).
+ * Supported: d in {32, 64, 128}; hq % hkv == 0; scale > 0 and finite.
+ *
+ * Pointers are DEVICE pointers into memory the caller owns; every tensor pointer must
+ * be 16-byte aligned.  The library never allocates or frees memory; scratch space is the
+ * caller's `workspace` (size from the *_workspace_size queries; it may be NULL when the
+ * size is 0).  `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ * call only enqueues work on it and returns without synchronising.
+ *
+ * Errors: arguments are validated on the host before anything is launched, so an
+ * ATTN_ERR_INVALID_ARG / ATTN_ERR_UNSUPPORTED return leaves every output untouched;
+ * attn_last_error_message() then says which argument was wrong.  A failed launch returns
+ * ATTN_ERR_CUDA.  Kernels never trap: a device-side problem (a pipeline wait that timed
+ * out, a sequence longer than max_seqlen) sets a per-device error word that
+ * attn_get_device_error() reads and clears.
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,   /* a pointer, size or shape argument is invalid          */
+    ATTN_ERR_UNSUPPORTED = 2,   /* valid but outside what this build supports (d, dtype) */
+    ATTN_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed                  */
+    ATTN_ERR_TIMEOUT = 4        /* a kernel's bounded pipeline wait ran out              */
+} attn_status;
+
+typedef enum {
+    ATTN_BF16 = 0,              /* bf16 tensors, fp32 accumulation (the fast path)       */
+    ATTN_FP32 = 1               /* fp32 tensors, fp32 arithmetic (numerical check mode)  */
+} attn_dtype;
+
+/* Forward.  Writes o [T,hq,d] and lse [hq,T].
+ * Defined by: tutorial sections 标准注意力三步 (the result), 分块 / Online Softmax 技巧
+ * (how it is reached) and 前向 (only O and the row statistics are stored). */
+attn_status attn_fwd(const void *q, const void *k, const void *v,
+                     const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
+                     int32_t max_seqlen, int32_t total_tokens,
+                     int32_t hq, int32_t hkv, int32_t d,
+                     float scale, int32_t causal, int32_t dtype,
+                     void *o, float *lse,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Backward.  Reads q, k, v, the forward's o and lse, and the upstream gradient dout;
+ * writes dq [T,hq,d], dk and dv [T,hkv,d] (dk/dv summed over each GQA group).
+ * Defined by: tutorial sections 反向 and 反向重算流程 (recompute S and P per tile from
+ * Q/K/V and the saved statistics, then form dQ/dK/dV from dO).
+ * Workspace (bf16 mode): D [hq,T] float32 and a float32 dQ accumulator [T,hq,d]. */
+attn_status attn_bwd(const void *q, const void *k, const void *v,
+                     const void *o, const void *dout, const float *lse,
+                     const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
+                     int32_t max_seqlen, int32_t total_tokens,
+                     int32_t hq, int32_t hkv, int32_t d,
+                     float scale, int32_t causal, int32_t dtype,
+                     void *dq, void *dk, void *dv,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes attn_fwd / attn_bwd need for these shape arguments (0 = none). */
+size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,
+                               int32_t hq, int32_t hkv, int32_t d, int32_t dtype);
+size_t attn_bwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,
+                               int32_t hq, int32_t hkv, int32_t d, int32_t dtype);
+
+/* Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns ATTN_OK, ATTN_ERR_TIMEOUT, ATTN_ERR_INVALID_ARG (max_seqlen too small) or
+ * ATTN_ERR_CUDA (the synchronisation itself failed). */
+attn_status attn_get_device_error(void *stream);
+
+/* Static description of a status code. */
+const char *attn_status_string(attn_status status);
+
+/* Human-readable reason for the last non-OK return on the calling thread ("" if none). */
+const char *attn_last_error_message(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */

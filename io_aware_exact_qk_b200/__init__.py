@@ -1,0 +1,160 @@
+"""io_aware_exact_qk_b200 -- exact scaled-dot-product attention on one B200 (sm_100a).
+
+A thin ctypes binding over ``libattn.so`` (declared in ``include/attn.h``).  The functions
+carry the C ABI's names and only marshal arguments: tensors are PyTorch device tensors
+(PyTorch is used for device memory and streams), every step of the computation runs in
+the library's CUDA kernels, and there is no CPU or library fallback -- if the shared
+library is missing or fails to load, every call raises.
+
+    o, lse = attn_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, scale=None, causal=False)
+    dq, dk, dv = attn_bwd(q, k, v, o, do, lse, ...)
+
+Layouts: q, o, do, dq ``[T, Hq, d]``; k, v, dk, dv ``[T, Hkv, d]``; lse ``[Hq, T]`` fp32;
+cu_seqlens int32 ``[B+1]`` on the device (varlen), or ``None`` with ``batch`` equal-length
+sequences of ``T // batch`` tokens.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+ATTN_BF16, ATTN_FP32 = 0, 1
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+def load_library():
+    """Load libattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIBRARY_PATH):
+        raise RuntimeError(f"{LIBRARY_PATH} is missing; build it with `python -m io_aware_exact_qk_b200.build`")
+    lib = ctypes.CDLL(LIBRARY_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32, vp, vp, vp, sz, vp]
+    lib.attn_fwd.restype = ctypes.c_int
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                             vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd.restype = ctypes.c_int
+    for name in ("attn_fwd_workspace_size", "attn_bwd_workspace_size"):
+        fn = getattr(lib, name)
+        fn.argtypes = [i32] * 7
+        fn.restype = sz
+    lib.attn_get_device_error.argtypes = [vp]
+    lib.attn_get_device_error.restype = ctypes.c_int
+    lib.attn_status_string.argtypes = [ctypes.c_int]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_last_error_message.argtypes = []
+    lib.attn_last_error_message.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status):
+    if status != ATTN_OK:
+        lib = load_library()
+        msg = lib.attn_last_error_message().decode() or lib.attn_status_string(status).decode()
+        raise AttnError(status, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_FP32
+    raise AttnError(ATTN_ERR_UNSUPPORTED, f"dtype {t.dtype} is not supported (bf16, or fp32 check mode)")
+
+
+def _shape_args(q, k, cu_seqlens, max_seqlen, batch):
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if cu_seqlens is None:
+        batch = 1 if batch is None else int(batch)
+        seqlen = T // batch if batch > 0 else 0
+        max_seqlen = seqlen
+    else:
+        batch = cu_seqlens.numel() - 1
+        seqlen = 0
+        if max_seqlen is None:
+            raise AttnError(ATTN_ERR_INVALID_ARG, "varlen calls need max_seqlen")
+    return batch, seqlen, int(max_seqlen), T, hq, hkv, d
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def workspace_size(kind, q, k, cu_seqlens=None, max_seqlen=None, batch=None):
+    """Bytes of workspace attn_fwd ("fwd") or attn_bwd ("bwd") needs."""
+    lib = load_library()
+    b, _, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    fn = lib.attn_fwd_workspace_size if kind == "fwd" else lib.attn_bwd_workspace_size
+    return int(fn(b, ms, T, hq, hkv, d, _dtype_code(q)))
+
+
+def attn_fwd(q, k, v, cu_seqlens=None, max_seqlen=None, scale=None, causal=False, batch=None,
+             o=None, lse=None, workspace=None, stream=None):
+    """Forward.  Returns (o [T,Hq,d], lse [Hq,T] fp32)."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(hq, T, dtype=torch.float32, device=q.device)
+    ws = workspace_size("fwd", q, k, cu_seqlens, max_seqlen, batch)
+    if ws and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), b, seqlen, ms, T, hq, hkv, d,
+                        float(scale), int(bool(causal)), _dtype_code(q), _ptr(o), _ptr(lse),
+                        _ptr(workspace), ws if workspace is not None else 0, _stream(stream)))
+    return o, lse
+
+
+def attn_bwd(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scale=None, causal=False, batch=None,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward.  Returns (dq [T,Hq,d], dk [T,Hkv,d], dv [T,Hkv,d])."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = workspace_size("bwd", q, k, cu_seqlens, max_seqlen, batch)
+    if ws and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _check(lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(cu_seqlens), b, seqlen,
+                        ms, T, hq, hkv, d, float(scale), int(bool(causal)), _dtype_code(q), _ptr(dq), _ptr(dk),
+                        _ptr(dv), _ptr(workspace), ws if workspace is not None else 0, _stream(stream)))
+    return dq, dk, dv
+
+
+def attn_get_device_error(stream=None):
+    """Synchronise the stream and raise if a kernel reported a device-side error."""
+    _check(load_library().attn_get_device_error(_stream(stream)))
+
+
+def attn_version():
+    return int(load_library().attn_version())

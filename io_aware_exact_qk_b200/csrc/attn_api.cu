@@ -1,0 +1,223 @@
+// attn_api.cu -- the C ABI declared in include/attn.h: argument validation on the host,
+// TMA descriptor encoding, dispatch to the kernels, and the per-device error word.
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace attn {
+
+__device__ uint32_t g_device_error = 0;
+
+namespace {
+
+thread_local char g_last_error[256] = {0};
+
+attn_status fail(attn_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+attn_status ok() {
+  g_last_error[0] = 0;
+  return ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared validation of the shape arguments; fills `pb`.
+attn_status check_shapes(const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                         int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                         int32_t dtype, Problem* pb) {
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return fail(ATTN_ERR_UNSUPPORTED, "dtype %d is not supported", dtype);
+  if (d != 32 && d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {32, 64, 128}", d);
+  if (hq <= 0 || hkv <= 0) return fail(ATTN_ERR_INVALID_ARG, "head counts must be positive (hq=%d hkv=%d)", hq, hkv);
+  if (hq % hkv != 0) return fail(ATTN_ERR_UNSUPPORTED, "hq=%d is not a multiple of hkv=%d", hq, hkv);
+  if (hq > 65535 || batch > 65535) return fail(ATTN_ERR_UNSUPPORTED, "hq and batch must be <= 65535");
+  if (batch < 0 || total_tokens < 0 || max_seqlen < 0)
+    return fail(ATTN_ERR_INVALID_ARG, "negative batch / total_tokens / max_seqlen");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (cu_seqlens == nullptr) {
+    if (seqlen < 0) return fail(ATTN_ERR_INVALID_ARG, "negative seqlen");
+    if ((int64_t)batch * seqlen != total_tokens)
+      return fail(ATTN_ERR_INVALID_ARG, "batch mode needs total_tokens == batch * seqlen (%d * %d != %d)", batch,
+                  seqlen, total_tokens);
+    max_seqlen = seqlen;
+  } else {
+    if (!aligned16(cu_seqlens) && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+      return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    if (max_seqlen > total_tokens) return fail(ATTN_ERR_INVALID_ARG, "max_seqlen > total_tokens");
+  }
+  // TMA row coordinates and the [hq, T] statistics are addressed with 32-bit rows.
+  if ((int64_t)total_tokens * hq > (int64_t)INT32_MAX * 4)
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+  pb->cu_seqlens = cu_seqlens;
+  pb->batch = batch;
+  pb->seqlen = cu_seqlens ? 0 : seqlen;
+  pb->max_seqlen = max_seqlen;
+  pb->total_tokens = total_tokens;
+  pb->hq = hq;
+  pb->hkv = hkv;
+  pb->d = d;
+  pb->scale = scale;
+  pb->causal = causal;
+  return ATTN_OK;
+}
+
+attn_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(ATTN_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(ATTN_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return ATTN_OK;
+}
+
+attn_status from_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle swz = box_inner * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : box_inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = enc(reinterpret_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                     int32_t seqlen, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d,
+                     float scale, int32_t causal, int32_t dtype, void* o, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  Problem pb;
+  attn_status st = check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal,
+                                dtype, &pb);
+  if (st != ATTN_OK) return st;
+  if (total_tokens == 0 || batch == 0) return ok();
+  if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+      (st = check_ptr(o, "o")) || (st = check_ptr(lse, "lse")))
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == ATTN_BF16)
+    return from_cuda(launch_fwd_bf16(pb, q, k, v, o, lse, s), "attn_fwd launch");
+  return from_cuda(launch_fwd_fp32(pb, static_cast<const float*>(q), static_cast<const float*>(k),
+                                   static_cast<const float*>(v), static_cast<float*>(o), lse, s),
+                   "attn_fwd (fp32 check mode) launch");
+}
+
+size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
+                               int32_t d, int32_t dtype) {
+  (void)batch, (void)max_seqlen, (void)total_tokens, (void)hq, (void)hkv, (void)d, (void)dtype;
+  return 0;
+}
+
+size_t attn_bwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
+                               int32_t d, int32_t dtype) {
+  Problem pb{};
+  pb.batch = batch;
+  pb.max_seqlen = max_seqlen;
+  pb.total_tokens = total_tokens;
+  pb.hq = hq;
+  pb.hkv = hkv;
+  pb.d = d;
+  if (total_tokens <= 0 || hq <= 0) return 0;
+  return dtype == ATTN_FP32 ? bwd_fp32_workspace_bytes(pb) : bwd_bf16_workspace_bytes(pb);
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                     int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                     int32_t dtype, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  Problem pb;
+  attn_status st = check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal,
+                                dtype, &pb);
+  if (st != ATTN_OK) return st;
+  if (total_tokens == 0 || batch == 0) return ok();
+  if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+      (st = check_ptr(o, "o")) || (st = check_ptr(dout, "dout")) || (st = check_ptr(lse, "lse")) ||
+      (st = check_ptr(dq, "dq")) || (st = check_ptr(dk, "dk")) || (st = check_ptr(dv, "dv")))
+    return st;
+  const size_t need = attn_bwd_workspace_size(batch, pb.max_seqlen, total_tokens, hq, hkv, d, dtype);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if (need > 0 && (st = check_ptr(workspace, "workspace"))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == ATTN_BF16)
+    return from_cuda(launch_bwd_bf16(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, s), "attn_bwd launch");
+  return from_cuda(launch_bwd_fp32(pb, static_cast<const float*>(q), static_cast<const float*>(k),
+                                   static_cast<const float*>(v), static_cast<const float*>(o),
+                                   static_cast<const float*>(dout), lse, static_cast<float*>(dq),
+                                   static_cast<float*>(dk), static_cast<float*>(dv), workspace, s),
+                   "attn_bwd (fp32 check mode) launch");
+}
+
+attn_status attn_get_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return from_cuda(e, "stream synchronize");
+  uint32_t word = 0;
+  const uint32_t zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof word);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+  if (e != cudaSuccess) return from_cuda(e, "reading the device error word");
+  if (word & ATTN_DEVERR_TIMEOUT) return fail(ATTN_ERR_TIMEOUT, "a kernel's pipeline wait timed out");
+  if (word & ATTN_DEVERR_SEQLEN) return fail(ATTN_ERR_INVALID_ARG, "a sequence is longer than max_seqlen");
+  return ok();
+}
+
+const char* attn_status_string(attn_status status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* attn_last_error_message(void) { return g_last_error; }
+
+int32_t attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,597 @@
+// bwd_sm100.cu -- exact attention backward for sm_100a (bf16 tensors): TMA + tcgen05.
+//
+// What it computes (the analytic gradient of O = softmax(scale Q K^T [+mask]) V):
+//     D_i   = sum_c dO_ic O_ic
+//     P_ij  = exp(scale S_ij - LSE_i),   S = Q K^T      (recomputed, never stored)
+//     dS_ij = P_ij (dO_i . V_j - D_i)
+//     dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO
+// The "FlashAttention 与高效注意力内核" tutorial, sections 反向 and 反向重算流程: the
+// backward reloads Q/K/V tiles, recomputes S and P on chip from the saved statistics,
+// combines them with dO, and drops every tile when it is done, so memory stays O(N).
+//
+// Three launches on the caller's stream:
+//   1. bwd_preprocess   D = rowsum(dO o O) into the workspace and zero the fp32 dQ
+//                       accumulator (HBM-bound).
+//   2. bwd_main         one CTA per (128-key tile, kv head, sequence).  The CTA keeps
+//                       K_j, V_j in shared memory and dK_j, dV_j in TMEM, and walks the
+//                       query tiles of every query head of its GQA group (so dK/dV need
+//                       no atomics).  Per query tile i (BM rows):
+//                         S^T  = K_j Q_i^T            (tcgen05, TMEM fp32)
+//                         dP^T = V_j dO_i^T           (tcgen05, TMEM fp32)
+//                         P^T, dS^T on the compute warpgroup, one key row per thread,
+//                           written back as bf16 over S^T / dP^T, dS^T also to SMEM
+//                         dV  += P^T dO_i             (A from TMEM)
+//                         dK  += dS^T Q_i             (A from TMEM)
+//                         dQ_i partial                (A, B from SMEM)
+//                       and a drain warpgroup adds each dQ_i partial into the fp32
+//                       accumulator with fp32 atomics (L2 reductions), reading it from a
+//                       double-buffered TMEM slot so the tensor core never waits on it.
+//   3. bwd_dq_convert   dQ = bf16(scale * accumulator) (HBM-bound).
+//
+// dQ strategy.  Each (key tile, query tile) pair contributes a BM x d partial of dQ_i;
+// the CTA that owns the key tile adds it into an fp32 accumulator with atomics.  The
+// alternative -- a second, query-major kernel -- would recompute S and dP (7 matrix
+// products per tile instead of 5, 40% more tensor work); the atomic traffic instead goes
+// to L2 (the accumulator of one head, N*d*4 bytes, stays L2-resident), coalesced
+// 128 bytes per warp instruction (d = 128) or 16-byte vector atomics (d <= 64).
+//
+// TMEM shapes.  d = 128 uses BM = 64 query rows per step and forms the transpose
+// dQ_i^T = K_j^T dS^T (M = d = 128, N = 64), which fits S^T (64) + dP^T (64) + dV (128)
+// + dK (128) + two dQ^T buffers (2 x 64) = 512 columns.  d <= 64 uses BM = 128 and
+// dQ_i = dS K_j (M = 128 query rows, N = d): 128 + 128 + 4 d <= 512 columns.
+//
+// Warp roles (320 threads): warps 0-3 compute (P^T, dS^T, epilogue of dK/dV), warps 4-7
+// dQ drain, warp 8 TMA producer (+ LSE / D rows into SMEM), warp 9 MMA issuer.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kKeys = 128;   // keys per CTA == TMEM lanes
+constexpr int kThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr bool DQT = (D == 128);          // dQ^T form (see file comment)
+  static constexpr int BM = DQT ? 64 : 128;       // query rows per step
+  static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span of Q/K/V/dO rows (bytes)
+  static constexpr int PANEL = SW / 2;
+  static constexpr int NPANEL = D / PANEL;
+  static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;
+  static constexpr int SBO = 8 * SW;
+  static constexpr int KSTEPS_PER_PANEL = SW / 32;
+  static constexpr int KV_PANEL_BYTES = kKeys * SW;   // panel of a 128-row K or V tile
+  static constexpr int KV_TILE_BYTES = kKeys * D * 2;
+  static constexpr int Q_PANEL_BYTES = BM * SW;       // panel of a BM-row Q or dO tile
+  static constexpr int Q_TILE_BYTES = BM * D * 2;
+  static constexpr int DS_PANEL_BYTES = kKeys * 128;  // dS^T: 128 key rows x 64 queries (bf16)
+  static constexpr int DS_BYTES = kKeys * BM * 2;
+  // TMEM columns
+  static constexpr int T_ST = 0;
+  static constexpr int T_DPT = BM;
+  static constexpr int T_DV = 2 * BM;
+  static constexpr int T_DK = 2 * BM + D;
+  static constexpr int T_DQ = 2 * BM + 2 * D;        // two buffers of DQ_COLS
+  static constexpr int DQ_COLS = DQT ? BM : D;
+  // shared memory map (offsets from the 1024-aligned base)
+  static constexpr int O_K = 0;
+  static constexpr int O_V = O_K + KV_TILE_BYTES;
+  static constexpr int O_Q = O_V + KV_TILE_BYTES;          // 2 stages
+  static constexpr int O_DO = O_Q + 2 * Q_TILE_BYTES;      // 2 stages
+  static constexpr int O_DS = O_DO + 2 * Q_TILE_BYTES;     // 2 buffers
+  static constexpr int O_LSE = O_DS + 2 * DS_BYTES;        // 2 stages x BM floats (LSE * log2 e)
+  static constexpr int O_DD = O_LSE + 2 * BM * 4;          // 2 stages x BM floats (D)
+  static constexpr int O_BAR = O_DD + 2 * BM * 4;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QFULL = 1;     // 2
+  static constexpr int B_QEMPTY = 3;    // 2
+  static constexpr int B_ST = 5;
+  static constexpr int B_DPT = 6;
+  static constexpr int B_PT = 7;
+  static constexpr int B_DS = 8;
+  static constexpr int B_DSFREE = 9;    // 2
+  static constexpr int B_DQFULL = 11;   // 2
+  static constexpr int B_DQEMPTY = 13;  // 2
+  static constexpr int B_DONE = 15;
+  static constexpr int NBARS = 16;
+  static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 16;
+};
+
+struct BwdParams {
+  const int32_t* cu_seqlens;
+  int32_t seqlen, max_seqlen, total_tokens, hq, hkv;
+  float scale;
+  float scale_log2;
+  int32_t causal;
+  const float* lse;      // [hq, T]
+  const float* dd;       // [hq, T]
+  float* dq_acc;         // [T, hq, d]
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+};
+
+// Enumerates the (query head, query tile) steps of one CTA in a fixed order.
+struct StepIter {
+  int G, i_begin, n_q, steps_per_head;
+  __device__ void head_tile(int n, int g, int* h, int* i) const {
+    *h = g * G + n / steps_per_head;
+    *i = i_begin + n % steps_per_head;
+  }
+};
+
+// Byte offset of the 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled panel.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                   const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int BM = C::BM;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  float* s_lse = reinterpret_cast<float*>(smem + C::O_LSE);
+  float* s_dd = reinterpret_cast<float*>(smem + C::O_DD);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::O_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x;        // kv head
+  const int b = blockIdx.y;        // sequence
+  const int jt = blockIdx.z;       // key tile (0 = most query tiles under causal: first)
+  const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
+  const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
+  const int kv0 = jt * kKeys;
+  if (kv0 >= len) return;
+  StepIter it;
+  it.G = p.hq / p.hkv;
+  it.n_q = (len + BM - 1) / BM;
+  it.i_begin = p.causal ? kv0 / BM : 0;
+  it.steps_per_head = it.n_q - it.i_begin;
+  const int n_steps = it.G * it.steps_per_head;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBARS; ++i) {
+      uint32_t cnt = 1;
+      if (i == C::B_QFULL || i == C::B_QFULL + 1) cnt = 32;
+      if (i == C::B_PT || i == C::B_DS || i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------- producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per step ----------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE_BYTES);
+      for (int pn = 0; pn < C::NPANEL; ++pn) {
+        tma_load_3d(sbase + C::O_K + pn * C::KV_PANEL_BYTES, &tmK, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
+        tma_load_3d(sbase + C::O_V + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
+      }
+    }
+    for (int n = 0; n < n_steps; ++n) {
+      const int s = n & 1;
+      if (!mbar_wait(bar(C::B_QEMPTY + s), ((n >> 1) & 1) ^ 1, abort_flag)) break;
+      int h, i;
+      it.head_tile(n, g, &h, &i);
+      const int q0 = i * BM;
+      for (int c = lane; c < BM; c += 32) {
+        const int qi = q0 + c;
+        const bool ok = qi < len;
+        const size_t idx = (size_t)h * p.total_tokens + seq_start + qi;
+        s_lse[s * BM + c] = ok ? p.lse[idx] * kLog2e : 0.f;
+        s_dd[s * BM + c] = ok ? p.dd[idx] : 0.f;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
+        for (int pn = 0; pn < C::NPANEL; ++pn) {
+          tma_load_3d(sbase + C::O_Q + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmQ, bar(C::B_QFULL + s),
+                      pn * C::PANEL, h, seq_start + q0);
+          tma_load_3d(sbase + C::O_DO + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmDO, bar(C::B_QFULL + s),
+                      pn * C::PANEL, h, seq_start + q0);
+        }
+      } else {
+        mbar_arrive(bar(C::B_QFULL + s));
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id_sdp = idesc_bf16_f32(kKeys, BM, false, false);   // K Q^T, V dO^T
+      const uint32_t id_grad = idesc_bf16_f32(kKeys, D, false, true);    // P^T dO, dS^T Q
+      const uint32_t id_dq = C::DQT ? idesc_bf16_f32(D, BM, true, true)  // K^T dS^T
+                                    : idesc_bf16_f32(BM, D, true, true); // dS K
+      auto kmajor_off = [&](int kk, int panel_bytes) {
+        return (uint32_t)((kk / C::KSTEPS_PER_PANEL) * panel_bytes + (kk % C::KSTEPS_PER_PANEL) * 32);
+      };
+      // X_tile (128 keys) times Y_i^T (BM rows), both K-major over d
+      auto issue_sdp = [&](uint32_t x_off, uint32_t y_off, uint32_t d_col) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = smem_desc(sbase + x_off + kmajor_off(kk, C::KV_PANEL_BYTES), 16, C::SBO, C::SWZ);
+          const uint64_t bd = smem_desc(sbase + y_off + kmajor_off(kk, C::Q_PANEL_BYTES), 16, C::SBO, C::SWZ);
+          mma_ss(tmem + d_col, a, bd, id_sdp, kk > 0 ? 1u : 0u);
+        }
+      };
+      // D[128 keys x d] += A^T(TMEM, bf16 over BM queries) * Y_i (BM x d, MN-major)
+      auto issue_grad = [&](uint32_t a_col, uint32_t y_off, uint32_t d_col, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint64_t bd = smem_desc(sbase + y_off + kk * 16 * C::SW, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
+          mma_ts(tmem + d_col, tmem + a_col + kk * 8, bd, id_grad, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto issue_dq = [&](int dsbuf, uint32_t d_col) {
+        const uint32_t ds = sbase + C::O_DS + dsbuf * C::DS_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t kdesc = smem_desc(sbase + C::O_K + kk * 16 * C::SW, C::KV_PANEL_BYTES, C::SBO, C::SWZ);
+          const uint64_t sdesc = smem_desc(ds + kk * 16 * 128, C::DS_PANEL_BYTES, 1024, 2u);
+          if (C::DQT)
+            mma_ss(tmem + d_col, kdesc, sdesc, id_dq, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + d_col, sdesc, kdesc, id_dq, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag) && mbar_wait(bar(C::B_QFULL), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(C::O_K, C::O_Q, C::T_ST);
+        mma_commit(bar(C::B_ST));
+        issue_sdp(C::O_V, C::O_DO, C::T_DPT);
+        mma_commit(bar(C::B_DPT));
+      }
+      for (int n = 0; ok && n < n_steps; ++n) {
+        const int s = n & 1;
+        const uint32_t q_off = C::O_Q + s * C::Q_TILE_BYTES;
+        const uint32_t do_off = C::O_DO + s * C::Q_TILE_BYTES;
+        const bool more = n + 1 < n_steps;
+        if (!mbar_wait(bar(C::B_PT), n & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_grad(C::T_ST, do_off, C::T_DV, n > 0);                  // dV += P^T dO
+        if (more) {
+          if (!mbar_wait(bar(C::B_QFULL + (s ^ 1)), ((n + 1) >> 1) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_sdp(C::O_K, C::O_Q + (s ^ 1) * C::Q_TILE_BYTES, C::T_ST);   // S^T for the next step
+          mma_commit(bar(C::B_ST));
+        }
+        if (!mbar_wait(bar(C::B_DS), n & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_grad(C::T_DPT, q_off, C::T_DK, n > 0);                  // dK += dS^T Q
+        mma_commit(bar(C::B_QEMPTY + s));
+        if (!mbar_wait(bar(C::B_DQEMPTY + s), ((n >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        issue_dq(s, C::T_DQ + s * C::DQ_COLS);                         // dQ_i partial
+        mma_commit(bar(C::B_DQFULL + s));
+        mma_commit(bar(C::B_DSFREE + s));
+        if (more) {
+          issue_sdp(C::O_V, C::O_DO + (s ^ 1) * C::Q_TILE_BYTES, C::T_DPT);  // dP^T for the next step
+          mma_commit(bar(C::B_DPT));
+        }
+      }
+      mma_commit(bar(C::B_DONE));
+    }
+  } else if (warp < 4) {
+    // ---------------- compute: P^T, dS^T (one key row per thread) ----------------
+    const int lane_base = warp * 32;
+    const int kr = lane_base + lane;              // key row inside the tile
+    const int kj = kv0 + kr;                      // key index inside the sequence
+    const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < n_steps; ++n) {
+      const int s = n & 1;
+      int h, i;
+      it.head_tile(n, g, &h, &i);
+      const int q0 = i * BM;
+      // visible query columns c: q0 + c < len, and (causal) q0 + c >= kj; key inside the sequence
+      int c_lo = 0, c_hi = BM;                    // [c_lo, c_hi)
+      if (q0 + BM > len) c_hi = len - q0;
+      if (p.causal && kj - q0 > c_lo) c_lo = kj - q0;
+      if (kj >= len) c_hi = 0;
+      if (!mbar_wait(bar(C::B_QFULL + s), (n >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_ST), n & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const float* lse = s_lse + s * BM;
+      const float* dd = s_dd + s * BM;
+      float pr[BM];
+#pragma unroll
+      for (int cb = 0; cb < BM; cb += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + C::T_ST + cb, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = cb + e;
+          const float x = fmaf(__uint_as_float(r[e]), sl2, -lse[c]);
+          pr[c] = (c >= c_lo && c < c_hi) ? ex2(x) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int cb = 0; cb < BM; cb += 32) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(pr[cb + 2 * e], pr[cb + 2 * e + 1]);
+        tmem_st16(trow + C::T_ST + cb / 2, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PT));
+      // dS^T = P^T o (dP^T - D): to TMEM (over dP^T) and to the swizzled SMEM buffer
+      if (!mbar_wait(bar(C::B_DSFREE + s), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_DPT), n & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint8_t* ds_smem = smem + C::O_DS + s * C::DS_BYTES;
+#pragma unroll
+      for (int cb = 0; cb < BM; cb += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + C::T_DPT + cb, r);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = cb + 2 * e;
+          const float d0 = pr[c] * (__uint_as_float(r[2 * e]) - dd[c]);
+          const float d1 = pr[c + 1] * (__uint_as_float(r[2 * e + 1]) - dd[c + 1]);
+          w[e] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(trow + C::T_DPT + cb / 2, w);
+        // queries cb..cb+31 live in panel cb/64, 16-byte chunks (cb%64)/8 .. +3
+        uint8_t* panel = ds_smem + (cb / 64) * C::DS_PANEL_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = (cb % 64) / 8 + ch;
+          *reinterpret_cast<uint4*>(panel + sw128_offset(kr, chunk)) =
+              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DS));
+    }
+    // ---------------- epilogue: dK = scale * acc, dV ----------------
+    if (ok && mbar_wait(bar(C::B_DONE), 0, abort_flag)) {
+      tc_fence_after();
+      const bool row_ok = kj < len;
+      const size_t orow = ((size_t)(seq_start + kj) * p.hkv + g) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
+        const float mul = which == 0 ? 1.f : p.scale;
+        const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t r[32];
+          tmem_ld32(trow + col + cb, r);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+            uint4* o4 = reinterpret_cast<uint4*>(dst + cb);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ---------------- dQ drain: TMEM partial -> fp32 atomics into the accumulator ---------
+    const int lane_base = (warp & 3) * 32;
+    const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
+    for (int n = 0; n < n_steps; ++n) {
+      const int s = n & 1;
+      int h, i;
+      it.head_tile(n, g, &h, &i);
+      const int q0 = i * BM;
+      if (!mbar_wait(bar(C::B_DQFULL + s), (n >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      uint32_t r[C::DQ_COLS / 32][32];
+#pragma unroll
+      for (int cb = 0; cb < C::DQ_COLS / 32; ++cb) tmem_ld32(trow + C::T_DQ + s * C::DQ_COLS + cb * 32, r[cb]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQEMPTY + s));
+      if (C::DQT) {
+        // lane = feature c, registers = the BM query rows of this step
+        const int c = lane_base + lane;
+        float* base = p.dq_acc + ((size_t)(seq_start + q0) * p.hq + h) * D + c;
+        const int rows = min(BM, len - q0);
+#pragma unroll
+        for (int e = 0; e < BM; ++e)
+          if (e < rows) atomicAdd(base + (size_t)e * p.hq * D, __uint_as_float(r[e / 32][e % 32]));
+      } else {
+        // lane = query row, registers = its d features (contiguous in memory)
+        const int qr = q0 + lane_base + lane;
+        if (qr < len) {
+          float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)(seq_start + qr) * p.hq + h) * D);
+#pragma unroll
+          for (int e = 0; e < D / 4; ++e)
+            atomicAdd(dst + e, make_float4(__uint_as_float(r[(4 * e) / 32][(4 * e) % 32]),
+                                           __uint_as_float(r[(4 * e + 1) / 32][(4 * e + 1) % 32]),
+                                           __uint_as_float(r[(4 * e + 2) / 32][(4 * e + 2) % 32]),
+                                           __uint_as_float(r[(4 * e + 3) / 32][(4 * e + 3) % 32])));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = sum_c dO_ic O_ic (fp32, from the stored bf16 O) and zero the dQ accumulator.
+// Each group of D/8 threads handles one (token, head) row with 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dout, int64_t rows, int hq,
+                                                      int total_tokens, float* __restrict__ dd,
+                                                      float* __restrict__ dq_acc) {
+  constexpr int TPR = D / 8;   // threads per row
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  // The loop condition is uniform over each warp (it tests the warp's first row), so the
+  // row-group shuffles below always run with all 32 lanes present.
+  const int64_t lane = threadIdx.x & 31;
+  for (int64_t base = tid; (base - lane) / TPR < rows; base += nthreads) {
+    const int64_t row = base / TPR;          // row = token * hq + head
+    const int part = (int)(base % TPR);
+    float acc = 0.f;
+    if (row < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+      const uint4 bb = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(a2[e]);
+        const float2 y = __bfloat1622float2(b2[e]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) {
+      const int64_t t = row / hq;
+      const int h = (int)(row % hq);
+      dd[(int64_t)h * total_tokens + t] = acc;
+    }
+  }
+}
+
+// dQ = bf16(scale * accumulator), 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ acc, int64_t n8, float scale,
+                                                      __nv_bfloat16* __restrict__ dq) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x * scale, a.y * scale);
+    w.y = pack_bf16x2(a.z * scale, a.w * scale);
+    w.z = pack_bf16x2(b.x * scale, b.y * scale);
+    w.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = w;
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                         cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  const size_t T = (size_t)pb.total_tokens;
+  float* dd = static_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           (((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255));
+  const int64_t rows = (int64_t)T * pb.hq;
+  {
+    const int64_t threads = rows * (D / 8);
+    const int blocks = (int)std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 16);
+    bwd_preprocess<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                   static_cast<const __nv_bfloat16*>(dout), rows, pb.hq,
+                                                   pb.total_tokens, dd, dq_acc);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  alignas(64) CUtensorMap tq, tk, tv, tdo;
+  if (!encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
+      !encode_tma_3d(&tdo, dout, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
+      !encode_tma_3d(&tk, k, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys) ||
+      !encode_tma_3d(&tv, v, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys))
+    return cudaErrorInvalidValue;
+  BwdParams p;
+  p.cu_seqlens = pb.cu_seqlens;
+  p.seqlen = pb.seqlen;
+  p.max_seqlen = pb.max_seqlen;
+  p.total_tokens = pb.total_tokens;
+  p.hq = pb.hq;
+  p.hkv = pb.hkv;
+  p.scale = pb.scale;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.causal = pb.causal;
+  p.lse = lse;
+  p.dd = dd;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  cudaError_t e = cudaFuncSetAttribute(bwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(pb.hkv, pb.batch, (pb.max_seqlen + kKeys - 1) / kKeys);
+  bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t n8 = rows * D / 8;
+  const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)sm_count() * 16);
+  bwd_dq_convert<<<blocks, 256, 0, stream>>>(dq_acc, n8, pb.scale, static_cast<__nv_bfloat16*>(dq));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_bf16_workspace_bytes(const Problem& pb) {
+  const size_t T = (size_t)pb.total_tokens;
+  const size_t dbytes = ((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255;   // D [hq, T]
+  const size_t qacc = T * (size_t)pb.hq * (size_t)pb.d * sizeof(float);             // dQ accumulator
+  return dbytes + qacc;
+}
+
+cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                            cudaStream_t stream) {
+  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
+  switch (pb.d) {
+    case 32: return launch_bwd_d<32>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
+    case 64: return launch_bwd_d<64>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
+    case 128: return launch_bwd_d<128>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,386 @@
+// fwd_sm100.cu -- exact attention forward for sm_100a: TMA + tcgen05 + TMEM.
+//
+// What it computes: O = softmax(scale * Q K^T [+ causal mask]) V and the per-row
+// LSE = m + ln l, for every (sequence, query head) ("FlashAttention 与高效注意力内核"
+// tutorial, sections 标准注意力三步 and 前向).
+//
+// How (sections 分块, Online Softmax 技巧 and 伪代码骨架 of the same tutorial; FA2's
+// query-outer loop order from the "Flash-Attention" concept page, 核心思想): each CTA owns
+// two 128-row query tiles of one head and streams the sequence's 128-key K/V tiles
+// through shared memory once.  Per key tile and query tile t:
+//     S_t   = Q_t K_j^T                  tcgen05 MMA, A and B from swizzled SMEM, fp32 in TMEM
+//     m_new = max(m_old, rowmax(S_t))    one query row per thread, no shuffles
+//     P_t   = exp2(S_t * scale*log2e - m_new), l = l * exp2(m_old - m_new) + rowsum(P_t)
+//     O_t   = exp2(m_old - m_new) * O_t + P_t V_j
+// with P_t stored as bf16 into the TMEM columns that held S_t and fed to the PV MMA
+// straight from TMEM.  The running O_t never leaves TMEM until the end, where it is
+// divided by l and written once with LSE (the tutorial's 前向: only O and the row
+// statistics reach HBM).
+//
+// Rescale skipping: m_new only moves when the tile max exceeds the running max by more
+// than 8 (in log2 units).  Otherwise the old max keeps being used, so P entries stay
+// <= 2^8 and O, l are left as they are; the final O / l and LSE use that same max
+// consistently, so the result is exact up to rounding.  (The concept page lists this
+// "conditional rescaling" among the Blackwell techniques, 已知局限.)
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + correction + epilogue for query tile 0 (TMEM lanes 0..127)
+//   warps 4-7  the same for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j / V_j into a STAGES-deep ring
+//   warp  9    MMA issuer (one thread): S0, S1, then PV0, S0', PV1, S1', ... so the tensor
+//              core works on one tile while the other tile's softmax runs.
+// TMEM (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 after.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kRows = 128;                 // query rows per tile == TMEM lanes
+constexpr int kKeys = 128;                 // keys per K/V tile
+constexpr float kRescaleSkip = 8.0f;       // log2 units, see file comment
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kThreads = 320;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int SW = D >= 64 ? 128 : 64;    // swizzle span == SMEM row pitch (bytes)
+  static constexpr int PANEL = SW / 2;             // bf16 elements per panel row
+  static constexpr int NPANEL = D / PANEL;         // panels per tile
+  static constexpr int PANEL_BYTES = kRows * SW;   // one panel of a 128-row tile
+  static constexpr int TILE_BYTES = kRows * D * 2;
+  static constexpr int STAGES = D == 128 ? 2 : (D == 64 ? 3 : 4);
+  static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;   // descriptor swizzle code
+  static constexpr int SBO = 8 * SW;               // bytes between 8-row swizzle atoms
+  static constexpr int KSTEPS_PER_PANEL = SW / 32; // 16-element K steps inside one panel
+  // barrier slots
+  static constexpr int B_Q = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_VFULL = B_KFULL + STAGES;
+  static constexpr int B_KEMPTY = B_VFULL + STAGES;
+  static constexpr int B_VEMPTY = B_KEMPTY + STAGES;
+  static constexpr int B_SFULL = B_VEMPTY + STAGES;  // 2
+  static constexpr int B_PFULL = B_SFULL + 2;        // 2
+  static constexpr int B_OFINAL = B_PFULL + 2;       // 2
+  static constexpr int NBARS = B_OFINAL + 2;
+  static constexpr int DATA_BYTES = (2 + 2 * STAGES) * TILE_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 16;
+};
+
+struct FwdParams {
+  const int32_t* cu_seqlens;
+  int32_t seqlen, max_seqlen, total_tokens, hq, hkv;
+  float scale_log2;  // scale * log2(e)
+  int32_t causal;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);   // 1024-aligned (swizzle atoms)
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + 2 * C::TILE_BYTES;
+  const uint32_t sV = sK + C::STAGES * C::TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
+  const int pair = gridDim.z - 1 - blockIdx.z;   // heaviest (last) query tiles first
+  const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
+  const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
+  if (len > p.max_seqlen) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) report_error(ATTN_DEVERR_SEQLEN);
+  }
+  const int q0 = pair * 2 * kRows;
+  if (q0 >= len) return;   // uniform over the CTA, before any barrier or TMEM use
+  const int kv_end = p.causal ? min(len, q0 + 2 * kRows) : len;
+  const int n_kv = (kv_end + kKeys - 1) / kKeys;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBARS; ++i) {
+      const bool per_thread = (i == C::B_PFULL || i == C::B_PFULL + 1);
+      mbar_init(bar(i), per_thread ? 128u : 1u);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const int hk = h / (p.hq / p.hkv);
+      mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int pn = 0; pn < C::NPANEL; ++pn)
+          tma_load_3d(sQ + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, bar(C::B_Q), pn * C::PANEL, h,
+                      seq_start + q0 + t * kRows);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        if (!mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
+        for (int pn = 0; pn < C::NPANEL; ++pn)
+          tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, hk,
+                      seq_start + j * kKeys);
+        if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
+        for (int pn = 0; pn < C::NPANEL; ++pn)
+          tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, hk,
+                      seq_start + j * kKeys);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(kRows, kKeys, false, false);  // Q, K both K-major
+      const uint32_t idesc_pv = idesc_bf16_f32(kRows, D, false, true);       // V is MN-major (d contiguous)
+      auto issue_qk = [&](int t, int s) {
+        const uint32_t d_tmem = tmem + t * kKeys;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / C::KSTEPS_PER_PANEL) * C::PANEL_BYTES + (kk % C::KSTEPS_PER_PANEL) * 32;
+          const uint64_t a = smem_desc(sQ + t * C::TILE_BYTES + off, 16, C::SBO, C::SWZ);
+          const uint64_t bd = smem_desc(sK + s * C::TILE_BYTES + off, 16, C::SBO, C::SWZ);
+          mma_ss(d_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool accumulate) {
+        const uint32_t d_tmem = tmem + 2 * kKeys + t * D;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint32_t a_tmem = tmem + t * kKeys + kk * 8;   // 16 bf16 keys = 8 packed columns
+          const uint64_t bd = smem_desc(sV + s * C::TILE_BYTES + kk * 16 * C::SW, C::PANEL_BYTES, C::SBO, C::SWZ);
+          mma_ts(d_tmem, a_tmem, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag) && mbar_wait(bar(C::B_KFULL), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(bar(C::B_SFULL + 0));
+        issue_qk(1, 0);
+        mma_commit(bar(C::B_SFULL + 1));
+        mma_commit(bar(C::B_KEMPTY + 0));
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        const bool more = j + 1 < n_kv;
+        const int s1 = (j + 1) % C::STAGES;
+        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+        if (!mbar_wait(bar(C::B_VFULL + s), ph, abort_flag)) break;
+        if (!mbar_wait(bar(C::B_PFULL + 0), j & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(0, s, j > 0);
+        if (more) {
+          if (!mbar_wait(bar(C::B_KFULL + s1), ph1, abort_flag)) break;
+          tc_fence_after();
+          issue_qk(0, s1);
+          mma_commit(bar(C::B_SFULL + 0));
+        } else {
+          mma_commit(bar(C::B_OFINAL + 0));
+        }
+        if (!mbar_wait(bar(C::B_PFULL + 1), j & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(1, s, j > 0);
+        mma_commit(bar(C::B_VEMPTY + s));
+        if (more) {
+          issue_qk(1, s1);
+          mma_commit(bar(C::B_SFULL + 1));
+          mma_commit(bar(C::B_KEMPTY + s1));
+        } else {
+          mma_commit(bar(C::B_OFINAL + 1));
+        }
+      }
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue (one query row per thread) ---------
+    const int t = warp >> 2;                        // query tile of this warpgroup
+    const int lane_base = (warp & 3) * 32;          // TMEM lanes this warp may touch
+    const int qi = q0 + t * kRows + lane_base + lane;   // query index inside the sequence
+    const uint32_t tS = tmem + ((uint32_t)lane_base << 16) + t * kKeys;
+    const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + 2 * kKeys + t * D;
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY;   // running max in log2 units (possibly stale by < 8)
+    float l = 0.f;              // running sum of exp2(x - m_used)
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait(bar(C::B_SFULL + t), j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float s[kKeys];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tS + 0, r0);
+        tmem_ld32(tS + 32, r1);
+        tmem_ld32(tS + 64, r2);
+        tmem_ld32(tS + 96, r3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          s[c] = __uint_as_float(r0[c]);
+          s[32 + c] = __uint_as_float(r1[c]);
+          s[64 + c] = __uint_as_float(r2[c]);
+          s[96 + c] = __uint_as_float(r3[c]);
+        }
+      }
+      // mask: key kbase + c is visible iff it is inside the sequence and, when causal,
+      // not after this query.
+      const int kbase = j * kKeys;
+      int lim = len - 1 - kbase;
+      if (p.causal) lim = min(lim, qi - kbase);
+      if (lim < kKeys - 1) {
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c)
+          if (c > lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = mx * sl2;
+      float m_new = m_used;
+      if (m_cand > m_used + kRescaleSkip) m_new = m_cand;
+      const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
+      float rowsum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2(fmaf(s[2 * c], sl2, -m_sub));
+        const float p1 = ex2(fmaf(s[2 * c + 1], sl2, -m_sub));
+        rowsum += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+        tmem_st32(tS + 0, lo);
+        tmem_st32(tS + 32, hi);
+      }
+      float alpha = 1.f;
+      if (m_new != m_used) {
+        alpha = ex2(m_used - m_sub);   // 0 when m_used is -inf
+        l = l * alpha + rowsum;
+      } else {
+        l += rowsum;
+      }
+      const bool need = (j > 0) && (m_new != m_used);
+      m_used = m_new;
+      if (__any_sync(0xffffffffu, need)) {
+        // O_t was last written by PV_t(j-1), which completed before S_t(j) was signalled.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(tO + c * 32, r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PFULL + t));
+    }
+    // ---------------- epilogue: O / l and LSE ----------------
+    if (ok && mbar_wait(bar(C::B_OFINAL + t), 0, abort_flag)) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const bool row_ok = qi < len;
+      __nv_bfloat16* orow = p.o + ((size_t)(seq_start + qi) * p.hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (row_ok) {
+        const float lse = l > 0.f ? (m_used == -INFINITY ? 0.f : m_used) * kLn2 + logf(l) : -INFINITY;
+        p.lse[(size_t)h * p.total_tokens + seq_start + qi] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const void* v, void* o, float* lse,
+                         cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  alignas(64) CUtensorMap tq, tk, tv;
+  if (!encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, kRows) ||
+      !encode_tma_3d(&tk, k, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys) ||
+      !encode_tma_3d(&tv, v, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys))
+    return cudaErrorInvalidValue;
+  FwdParams p;
+  p.cu_seqlens = pb.cu_seqlens;
+  p.seqlen = pb.seqlen;
+  p.max_seqlen = pb.max_seqlen;
+  p.total_tokens = pb.total_tokens;
+  p.hq = pb.hq;
+  p.hkv = pb.hkv;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.causal = pb.causal;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
+  dim3 grid(pb.hq, pb.batch, pairs);
+  fwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, void* o, float* lse,
+                            cudaStream_t stream) {
+  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
+  switch (pb.d) {
+    case 32: return launch_fwd_d<32>(pb, q, k, v, o, lse, stream);
+    case 64: return launch_fwd_d<64>(pb, q, k, v, o, lse, stream);
+    case 128: return launch_fwd_d<128>(pb, q, k, v, o, lse, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,45 @@
+// kernels.h -- internal launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace attn {
+
+// One attention problem as described by the C ABI's shape arguments.
+struct Problem {
+  const int32_t* cu_seqlens;  // device prefix sums [batch + 1], or nullptr for batch mode
+  int32_t batch;              // number of sequences
+  int32_t seqlen;             // batch mode: tokens per sequence
+  int32_t max_seqlen;         // >= every sequence length
+  int32_t total_tokens;       // T
+  int32_t hq, hkv, d;
+  float scale;
+  int32_t causal;
+};
+
+// Forward, bf16 tensors (tcgen05 path).  o [T,hq,d] bf16, lse [hq,T] f32.
+cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, void* o,
+                            float* lse, cudaStream_t stream);
+
+// Backward, bf16 tensors (tcgen05 path).  Workspace: bwd_bf16_workspace_bytes(pb).
+size_t bwd_bf16_workspace_bytes(const Problem& pb);
+cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                            cudaStream_t stream);
+
+// fp32 check mode (SIMT fp32 arithmetic).
+cudaError_t launch_fwd_fp32(const Problem& pb, const float* q, const float* k, const float* v, float* o,
+                            float* lse, cudaStream_t stream);
+size_t bwd_fp32_workspace_bytes(const Problem& pb);
+cudaError_t launch_bwd_fp32(const Problem& pb, const float* q, const float* k, const float* v, const float* o,
+                            const float* dout, const float* lse, float* dq, float* dk, float* dv, void* workspace,
+                            cudaStream_t stream);
+
+// Host helper shared by the launchers: encodes a 3-D bf16 TMA descriptor over a
+// [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that
+// matches a box_inner * 2-byte row (128 B or 64 B).
+bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows);
+
+}  // namespace attn

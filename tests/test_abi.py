@@ -1,0 +1,88 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/attn.h
+declares, and rejects bad arguments on the host before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_exact_qk_b200 as attn
+from io_aware_exact_qk_b200 import build as attn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    attn_build.build()
+    return attn.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert {"attn_fwd", "attn_bwd", "attn_fwd_workspace_size", "attn_bwd_workspace_size",
+            "attn_get_device_error", "attn_status_string", "attn_last_error_message", "attn_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.attn_status_string(0) == b"ok"
+    assert lib.attn_status_string(4) == b"device pipeline wait timed out"
+    assert attn.attn_version() == 100
+
+
+def _fwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, cu=None, batch=1, seqlen=8, max_seqlen=8, total=8, hq=2, hkv=2, d=64,
+             scale=0.125, causal=0, dtype=0, o=16, lse=16, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return lib.attn_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["cu"]), a["batch"], a["seqlen"],
+                        a["max_seqlen"], a["total"], a["hq"], a["hkv"], a["d"], a["scale"], a["causal"],
+                        a["dtype"], vp(a["o"]), vp(a["lse"]), vp(a["ws"]), a["wsb"], vp(a["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(hq=3, hkv=2), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(hq=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(dtype=7), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(total=9), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(q=None), attn.ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), attn.ATTN_ERR_INVALID_ARG),
+    (dict(o=0x1008), attn.ATTN_ERR_INVALID_ARG),
+    (dict(batch=-1, total=-8), attn.ATTN_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_arguments_on_host(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+    assert lib.attn_last_error_message() != b""
+
+
+def test_empty_problem_is_a_no_op(lib):
+    assert _fwd(lib, batch=0, seqlen=8, total=0, q=None, k=None, v=None, o=None, lse=None) == attn.ATTN_OK
+    assert _fwd(lib, batch=3, seqlen=0, total=0, q=None, k=None, v=None, o=None, lse=None) == attn.ATTN_OK
+
+
+def test_bwd_rejects_small_workspace(lib):
+    vp = ctypes.c_void_p
+    need = lib.attn_bwd_workspace_size(1, 8, 8, 2, 2, 64, 0)
+    assert need == ((2 * 8 * 4 + 255) // 256) * 256 + 8 * 2 * 64 * 4
+    st = lib.attn_bwd(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), None, 1, 8, 8, 8, 2, 2, 64, 0.125, 0, 0,
+                      vp(16), vp(16), vp(16), vp(16), need - 1, None)
+    assert st == attn.ATTN_ERR_INVALID_ARG
+    assert b"workspace" in lib.attn_last_error_message()
+
+
+def test_workspace_sizes(lib):
+    assert lib.attn_fwd_workspace_size(4, 2048, 8192, 16, 16, 128, 0) == 0
+    assert lib.attn_bwd_workspace_size(1, 0, 0, 4, 4, 64, 0) == 0
+    assert lib.attn_bwd_workspace_size(2, 10, 20, 4, 2, 32, 1) == 4 * 20 * 4   # fp32 mode: D only

@@ -1,0 +1,77 @@
+"""GPU parity of the backward (tcgen05 bf16 path and fp32 check mode) against the fp64 oracle.
+
+The GPU backward consumes the GPU forward's O and LSE, as a caller would; the oracle
+forms its own from the definition."""
+import numpy as np
+import pytest
+import torch
+
+import attn_workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, dtype=torch.bfloat16):
+    q, k, v, do, cu = W.make_inputs(w, dtype=dtype)
+    o, lse = P.gpu_fwd(w, q, k, v, cu)
+    grads = P.gpu_bwd(w, q, k, v, o.cpu(), do, lse.cpu(), cu)
+    ref = P.oracle_bwd(w, q, k, v, do, cu)
+    return grads, ref
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_small_config(causal):
+    w = W.small(causal)
+    grads, ref = _run(w)
+    P.check_grads_bf16(grads, ref[:3], tag=w.name)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ragged_varlen_gqa(d, causal):
+    """Lengths around the 64/128-row tile edges, one empty sequence, GQA 8:2."""
+    w = W.custom(f"ragged_d{d}", [1, 63, 64, 65, 127, 128, 129, 0, 200, 383], 8, 2, d, causal, seed=40 + d)
+    grads, ref = _run(w)
+    P.check_grads_bf16(grads, ref[:3], tag=w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mha2k_config(causal):
+    w = W.mha2k(causal)
+    grads, ref = _run(w)
+    P.check_grads_bf16(grads, ref[:3], tag=w.name)
+
+
+def test_mqa_batch_mode():
+    w = W.Workload("mqa", 2, 520, 4, 1, 128, True, seed=78)
+    grads, ref = _run(w)
+    P.check_grads_bf16(grads, ref[:3], tag=w.name)
+
+
+def test_gradient_sums_at_size():
+    """Properties that hold at any size: per (sequence, kv head) sum_j dK_j = 0 and
+    sum_j dV_j = sum over the group's query heads and rows of dO."""
+    w = W.custom("sums", [3000, 1100], 8, 2, 128, True, seed=79)
+    q, k, v, do, cu = W.make_inputs(w)
+    o, lse = P.gpu_fwd(w, q, k, v, cu)
+    dq, dk, dv = P.gpu_bwd(w, q, k, v, o.cpu(), do, lse.cpu(), cu)
+    dk, dv, dof = P.to_np(dk), P.to_np(dv), do.double().numpy()
+    G = w.hq // w.hkv
+    for bi in range(2):
+        sl = slice(int(cu[bi]), int(cu[bi + 1]))
+        sk = dk[sl].sum(axis=0)
+        assert np.abs(sk).max() <= 2e-2 * np.abs(dk[sl]).sum(axis=0).max()
+        want = dof[sl].reshape(-1, w.hkv, G, w.d).sum(axis=(0, 2))
+        assert P.rel_l2(dv[sl].sum(axis=0), want) < 1e-2
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp32_check_mode(d, causal):
+    w = W.custom(f"fp32b_d{d}", [1, 77, 150], 4, 2, d, causal, seed=60 + d)
+    grads, ref = _run(w, dtype=torch.float32)
+    for name, g, r in zip(("dq", "dk", "dv"), grads, ref[:3]):
+        g = P.to_np(g)
+        assert P.rel_l2(g, r) <= P.FP32_REL, name
+        assert P.max_rel(g, r) <= P.FP32_REL, name
