@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: attn_fwd and
+attn_bwd (D preprocess, main backward, dQ convert) on the multi-head workload
+B=4, H=16, N=2048, d=128, bf16, once without and once with the causal mask.  The metric is
+attention TFLOP/s (4*B*H*N^2*d for the forward, 2.5x that for the backward, halved for
+causal) and its fraction of the measured dense BF16 tensor-core peak.
+
+One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE); each rank runs its own
+batch (weak scaling, no collective on the data path); the time is the max over ranks.
+Timing: CUDA events on the launching stream around each step, L2 flushed (a 256 MiB
+write) between timed steps, per-kernel times from the library's own launch events.
+``--impl reference`` times the fp64 CPU oracle (the only reference there is) on a bounded
+sample of the same workload, on rank 0 only.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import attn_workloads as W  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPs/s on 1 B200 (bf16, d=128) and % of dense BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+DATA = "synthetic: Q, K, V, dO iid N(0,1) drawn in fp32 from a seeded torch CPU generator, rounded to bf16"
+
+
+def workload_variants(rank=0):
+    base = W.mha2k(False)
+    base = W.Workload(base.name, base.batch, base.seqlen, base.hq, base.hkv, base.d, False, seed=base.seed + rank)
+    return [base, base.with_causal(True)]
+
+
+def config_block(n_gpus):
+    w = W.mha2k(False)
+    return {"workload": f"mha2k: B={w.batch} H={w.hq} N={w.seqlen} d={w.d} bf16, fwd+bwd, non-causal and causal",
+            "global_batch": w.batch * n_gpus, "seq_len": w.seqlen, "heads": w.hq, "head_dim": w.d,
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{n_gpus}"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"bf16_tflops": float(p["bf16_tflops"]), "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", 0)),
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that, keep going
+            self.err = str(e)
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self.stop_flag.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU side: the fp64 oracle as a timed baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------------------
+_ORACLE_CACHE = {}
+
+
+def oracle_sample(heads, budget_s=None):
+    """Oracle forward + backward on whole heads of sequence 0 of both variants.  Runs the
+    given number of heads, or (budget_s) adds heads until the budget is spent.
+    Returns (algorithmic flops, seconds, heads done, threads)."""
+    import oracle
+    flops, secs, done = 0.0, 0.0, 0
+    threads = oracle.default_threads()
+    base = workload_variants()[0]
+    if "inputs" not in _ORACLE_CACHE:
+        _ORACLE_CACHE["inputs"] = W.make_inputs(base)
+    q, k, v, do, _ = _ORACLE_CACHE["inputs"]
+    n = base.seqlen
+    for h in range(base.hq):
+        if heads is not None and done >= heads:
+            break
+        if budget_s is not None and secs >= budget_s:
+            break
+        sl = (slice(0, n), slice(h, h + 1))
+        qs, ks, vs, dos = (t[sl].contiguous() for t in (q, k, v, do))
+        for causal in (False, True):
+            t0 = time.perf_counter()
+            oracle.attn_fwd(qs, ks, vs, scale=base.scale, causal=causal, threads=threads)
+            oracle.attn_bwd(qs, ks, vs, dos, scale=base.scale, causal=causal, threads=threads)
+            secs += time.perf_counter() - t0
+            f = 4.0 * n * n * base.d * (0.5 if causal else 1.0)
+            flops += 3.5 * f
+        done += 1
+    return flops, secs, done, threads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(heads=1)
+    flops = secs = 0.0
+    threads = 1
+    for _ in range(args.steps):
+        f, s, _, threads = oracle_sample(heads=1)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    sample = "fp64 CPU oracle, fwd+bwd of 1 head (N=2048, d=128) of sequence 0, non-causal and causal, per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": config_block(world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU side
+# ---------------------------------------------------------------------------------------
+def traffic_record(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "io_aware_exact_qk_b200", "csrc", rec["source"])
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+
+
+def run_ours(args, rank, world, local_rank):
+    import io_aware_exact_qk_b200 as attn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    attn.load_library()
+    variants = workload_variants(rank)
+    q, k, v, do, _ = W.make_inputs(variants[0])
+    host = {"q": q.pin_memory(), "k": k.pin_memory(), "v": v.pin_memory(), "do": do.pin_memory()}
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    w0 = variants[0]
+    outs = {}
+    for w in variants:
+        outs[w.causal] = {"o": torch.empty_like(qd), "lse": torch.empty(w.hq, w.total_tokens, device=dev),
+                          "dq": torch.empty_like(qd), "dk": torch.empty_like(kd), "dv": torch.empty_like(vd)}
+    ws = torch.empty(attn.workspace_size("bwd", qd, kd, batch=w0.batch), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for w in variants:
+            b = outs[w.causal]
+            attn.attn_fwd(qd, kd, vd, scale=w.scale, causal=w.causal, batch=w.batch, o=b["o"], lse=b["lse"])
+            attn.attn_bwd(qd, kd, vd, b["o"], dod, b["lse"], scale=w.scale, causal=w.causal, batch=w.batch,
+                          dq=b["dq"], dk=b["dk"], dv=b["dv"], workspace=ws)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    flops_fwd = {w.causal: w.fwd_flops() for w in variants}
+    flops_step = sum(w.fwd_flops() + w.bwd_flops() for w in variants)
+
+    for _ in range(args.warmup):
+        step()
+    attn.attn_get_device_error()
+    barrier()
+
+    # ---- timed region (device): per-step events, L2 flushed between steps ----
+    attn.attn_profile_collect()
+    attn.attn_profile_enable(True)
+    launches0 = attn.attn_launch_count()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        for s, e in events:
+            flush.zero_()
+            s.record(stream)
+            step()
+            e.record(stream)
+        barrier()
+    attn.attn_profile_enable(False)
+    launches = attn.attn_launch_count() - launches0
+    per_kernel = attn.attn_profile_collect()
+    attn.attn_get_device_error()
+    total_ms = sum(s.elapsed_time(e) for s, e in events)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"quick": True, "value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
+                              "kernels": {k: list(v) for k, v in per_kernel.items()}, "gpu_launches": launches}))
+        return
+    e2e_bufs = {}
+    e2e_out = {}
+    for w in variants:
+        _, e2e_bufs[w.causal] = attn.attention_host(host["q"], host["k"], host["v"], host["do"], scale=w.scale,
+                                                    causal=w.causal, batch=w.batch)
+    torch.cuda.synchronize()
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "do")) * len(variants)
+    d2h = sum(b["host_" + n].numel() * b["host_" + n].element_size()
+              for b in e2e_bufs.values() for n in ("o", "lse", "dq", "dk", "dv"))
+    barrier()
+    e2e_start, e2e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_start.record(stream)
+    for _ in range(args.steps):
+        for w in variants:
+            e2e_out[w.causal], _ = attn.attention_host(host["q"], host["k"], host["v"], host["do"], scale=w.scale,
+                                                       causal=w.causal, batch=w.batch, out=e2e_bufs[w.causal])
+    e2e_end.record(stream)
+    barrier()
+    attn.attn_get_device_error()
+    e2e_ms = e2e_start.elapsed_time(e2e_end)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * flops_step * args.steps / (float(t.item()) / 1e3) / 1e12
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    # dominant kernel and its roofline (algorithmic FLOPs per launch / mean event duration)
+    dom = max(per_kernel, key=lambda n: per_kernel[n][0])
+    dom_ms, dom_n = per_kernel[dom]
+    if dom.startswith("bwd_bf16"):
+        dom_flops = sum(2.5 * f for f in flops_fwd.values()) * args.steps
+    else:
+        dom_flops = sum(flops_fwd.values()) * args.steps
+    achieved = dom_flops / (dom_ms / 1e3) / 1e12
+    traffic = traffic_record(dom)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": UNIT,
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} dense bf16 (burst)",
+                "flops_per_launch": dom_flops / dom_n, "mean_launch_ms": dom_ms / dom_n}
+    breakdown = {}
+    for name, (ms, n) in sorted(per_kernel.items()):
+        breakdown[name] = {"launches": n, "total_ms": ms, "share": ms / sum(x[0] for x in per_kernel.values())}
+    cpu = None
+    if world == 1:
+        f, s, heads, threads = oracle_sample(heads=None, budget_s=12.0)
+        cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 CPU oracle, fwd+bwd of {heads} whole head(s) (N=2048, d=128) of sequence 0, "
+                         f"non-causal and causal, {s:.1f} s"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config_block(world),
+            "pct_of_peak": value / peaks["bf16_tflops"], "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "clocks": clocks.summary(), "kernels": breakdown}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true",
+                    help="device timing only: skip the end-to-end loop and the CPU baseline (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -119,6 +119,20 @@ const char *attn_status_string(attn_status status);
 /* Human-readable reason for the last non-OK return on the calling thread ("" if none). */
 const char *attn_last_error_message(void);
 
+/* ---- launch timing (tracing) ----------------------------------------------------------
+ * Off by default.  While enabled, every kernel the library launches is bracketed by a
+ * pair of CUDA events recorded on the launch's stream.  attn_profile_collect()
+ * synchronises those events, adds each launch's duration (milliseconds) and count into
+ * total_ms[kind] / launches[kind] for kind < n, and forgets them.  Kinds are numbered
+ * 0 .. attn_profile_kernel_count() - 1 and named by attn_profile_kernel_name().
+ * attn_launch_count() counts every kernel launch since the library was loaded, enabled
+ * or not.  The event pool is owned by the library; nothing is allocated on the device. */
+attn_status attn_profile_enable(int32_t on);
+int32_t attn_profile_kernel_count(void);
+const char *attn_profile_kernel_name(int32_t kind);
+attn_status attn_profile_collect(double *total_ms, int64_t *launches, int32_t n);
+int64_t attn_launch_count(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int32_t attn_version(void);
 

@@ -60,6 +60,16 @@ def load_library():
     lib.attn_last_error_message.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []
     lib.attn_version.restype = i32
+    lib.attn_profile_enable.argtypes = [i32]
+    lib.attn_profile_enable.restype = ctypes.c_int
+    lib.attn_profile_kernel_count.argtypes = []
+    lib.attn_profile_kernel_count.restype = i32
+    lib.attn_profile_kernel_name.argtypes = [i32]
+    lib.attn_profile_kernel_name.restype = ctypes.c_char_p
+    lib.attn_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), i32]
+    lib.attn_profile_collect.restype = ctypes.c_int
+    lib.attn_launch_count.argtypes = []
+    lib.attn_launch_count.restype = ctypes.c_int64
     _lib = lib
     return lib
 
@@ -158,3 +168,59 @@ def attn_get_device_error(stream=None):
 
 def attn_version():
     return int(load_library().attn_version())
+
+
+def attn_profile_enable(on=True):
+    """Turn per-launch CUDA-event timing of the library's kernels on or off."""
+    _check(load_library().attn_profile_enable(int(bool(on))))
+
+
+def attn_profile_collect():
+    """{kernel name: (total ms, launches)} for the launches timed since the last collect."""
+    lib = load_library()
+    n = lib.attn_profile_kernel_count()
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(lib.attn_profile_collect(ms, cnt, n))
+    return {lib.attn_profile_kernel_name(i).decode(): (ms[i], cnt[i]) for i in range(n) if cnt[i]}
+
+
+def attn_launch_count():
+    """Kernel launches made by the library since it was loaded."""
+    return int(load_library().attn_launch_count())
+
+
+def attention_host(q, k, v, do, cu_seqlens=None, max_seqlen=None, scale=None, causal=False, batch=None,
+                   device=None, stream=None, out=None):
+    """Forward and backward on HOST tensors: copies q, k, v, do (ideally pinned) to the
+    device, runs attn_fwd and attn_bwd there, and copies O, LSE, dQ, dK, dV back into host
+    tensors.  Returns (o, lse, dq, dk, dv) on the host.  ``out`` may hold preallocated
+    device and pinned host buffers (a dict from a previous call) to avoid reallocation."""
+    device = torch.device("cuda") if device is None else device
+    bufs = out if out is not None else {}
+    if not bufs:
+        for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=device)
+        bufs["cu"] = None if cu_seqlens is None else torch.empty(cu_seqlens.shape, dtype=torch.int32, device=device)
+        T, hq, _ = q.shape
+        bufs["o"] = torch.empty_like(bufs["q"])
+        bufs["lse"] = torch.empty(hq, T, dtype=torch.float32, device=device)
+        bufs["dq"] = torch.empty_like(bufs["q"])
+        bufs["dk"] = torch.empty_like(bufs["k"])
+        bufs["dv"] = torch.empty_like(bufs["v"])
+        ws = max(workspace_size("fwd", q, k, cu_seqlens, max_seqlen, batch),
+                 workspace_size("bwd", q, k, cu_seqlens, max_seqlen, batch))
+        bufs["ws"] = torch.empty(max(ws, 1), dtype=torch.uint8, device=device)
+        for name in ("o", "lse", "dq", "dk", "dv"):
+            bufs["host_" + name] = torch.empty(bufs[name].shape, dtype=bufs[name].dtype, pin_memory=True)
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        bufs[name].copy_(t, non_blocking=True)
+    if cu_seqlens is not None:
+        bufs["cu"].copy_(cu_seqlens, non_blocking=True)
+    attn_fwd(bufs["q"], bufs["k"], bufs["v"], bufs["cu"], max_seqlen, scale, causal, batch,
+             o=bufs["o"], lse=bufs["lse"], stream=stream)
+    attn_bwd(bufs["q"], bufs["k"], bufs["v"], bufs["o"], bufs["do"], bufs["lse"], bufs["cu"], max_seqlen, scale,
+             causal, batch, dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], workspace=bufs["ws"], stream=stream)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        bufs["host_" + name].copy_(bufs[name], non_blocking=True)
+    return tuple(bufs["host_" + n] for n in ("o", "lse", "dq", "dk", "dv")), bufs

@@ -5,7 +5,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "../../include/attn.h"
 #include "kernels.h"
@@ -99,7 +101,57 @@ attn_status from_cuda(cudaError_t e, const char* what) {
   return fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// ---- launch bookkeeping ---------------------------------------------------------------
+struct EventPair {
+  cudaEvent_t start = nullptr, end = nullptr;
+  int kind = 0;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<EventPair> g_prof_pool;      // created events, reused
+std::vector<int> g_prof_pending;         // indices into the pool recorded since the last collect
+std::vector<int> g_prof_free;            // indices free for reuse
+std::atomic<int64_t> g_launches{0};
+
 }  // namespace
+
+const char* kernel_kind_name(int kind) {
+  static const char* names[K_NUM_KINDS] = {"fwd_bf16_sm100",  "bwd_preprocess",       "bwd_bf16_sm100",
+                                           "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",
+                                           "bwd_fp32_dkdv_kernel"};
+  return (kind >= 0 && kind < K_NUM_KINDS) ? names[kind] : "";
+}
+
+LaunchScope::LaunchScope(int k, cudaStream_t s) : kind(k), stream(s), slot(-1) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  int idx;
+  if (!g_prof_free.empty()) {
+    idx = g_prof_free.back();
+    g_prof_free.pop_back();
+  } else {
+    EventPair ep;
+    if (cudaEventCreate(&ep.start) != cudaSuccess || cudaEventCreate(&ep.end) != cudaSuccess) return;
+    g_prof_pool.push_back(ep);
+    idx = (int)g_prof_pool.size() - 1;
+  }
+  g_prof_pool[idx].kind = kind;
+  if (cudaEventRecord(g_prof_pool[idx].start, stream) != cudaSuccess) {
+    g_prof_free.push_back(idx);
+    return;
+  }
+  slot = idx;
+}
+
+LaunchScope::~LaunchScope() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (cudaEventRecord(g_prof_pool[slot].end, stream) == cudaSuccess)
+    g_prof_pending.push_back(slot);
+  else
+    g_prof_free.push_back(slot);
+}
 
 bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
@@ -217,6 +269,42 @@ const char* attn_status_string(attn_status status) {
 }
 
 const char* attn_last_error_message(void) { return g_last_error; }
+
+attn_status attn_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return ok();
+}
+
+int32_t attn_profile_kernel_count(void) { return K_NUM_KINDS; }
+
+const char* attn_profile_kernel_name(int32_t kind) { return kernel_kind_name(kind); }
+
+attn_status attn_profile_collect(double* total_ms, int64_t* launches, int32_t n) {
+  std::vector<int> pending;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    pending.swap(g_prof_pending);
+  }
+  attn_status st = ok();
+  for (int idx : pending) {
+    const EventPair& ep = g_prof_pool[idx];
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(ep.end);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, ep.start, ep.end);
+    if (e != cudaSuccess) {
+      st = from_cuda(e, "reading launch timing events");
+    } else if (ep.kind < n) {
+      if (total_ms) total_ms[ep.kind] += ms;
+      if (launches) launches[ep.kind] += 1;
+    }
+  }
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int idx : pending) g_prof_free.push_back(idx);
+  return st;
+}
+
+int64_t attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int32_t attn_version(void) { return 100; }
 

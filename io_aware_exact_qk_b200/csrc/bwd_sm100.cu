@@ -534,6 +534,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   {
     const int64_t threads = rows * (D / 8);
     const int blocks = (int)std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 16);
+    LaunchScope scope(K_BWD_PREPROCESS, stream);
     bwd_preprocess<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                    static_cast<const __nv_bfloat16*>(dout), rows, pb.hq,
                                                    pb.total_tokens, dd, dq_acc);
@@ -564,11 +565,15 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   cudaError_t e = cudaFuncSetAttribute(bwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(pb.hkv, pb.batch, (pb.max_seqlen + kKeys - 1) / kKeys);
-  bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
-  e = cudaGetLastError();
+  {
+    LaunchScope scope(K_BWD_BF16, stream);
+    bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   const int64_t n8 = rows * D / 8;
   const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)sm_count() * 16);
+  LaunchScope scope(K_BWD_DQ_CONVERT, stream);
   bwd_dq_convert<<<blocks, 256, 0, stream>>>(dq_acc, n8, pb.scale, static_cast<__nv_bfloat16*>(dq));
   return cudaGetLastError();
 }

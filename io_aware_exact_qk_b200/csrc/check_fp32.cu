@@ -254,6 +254,7 @@ template <int D>
 cudaError_t fwd_fp32_d(const Problem& pb, const float* q, const float* k, const float* v, float* o, float* lse,
                        cudaStream_t st) {
   dim3 grid((pb.max_seqlen + kRowsPerBlock - 1) / kRowsPerBlock, pb.hq, pb.batch);
+  LaunchScope scope(K_FWD_FP32, st);
   fwd_fp32_kernel<D><<<grid, 256, 0, st>>>(q, k, v, pb, o, lse);
   return cudaGetLastError();
 }
@@ -263,10 +264,15 @@ cudaError_t bwd_fp32_d(const Problem& pb, const float* q, const float* k, const 
                        const float* dout, const float* lse, float* dq, float* dk, float* dv, float* dd,
                        cudaStream_t st) {
   dim3 g1((pb.max_seqlen + kRowsPerBlock - 1) / kRowsPerBlock, pb.hq, pb.batch);
-  bwd_fp32_dq_kernel<D><<<g1, 256, 0, st>>>(q, k, v, o, dout, lse, pb, dq, dd);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  {
+    LaunchScope scope(K_BWD_FP32_DQ, st);
+    bwd_fp32_dq_kernel<D><<<g1, 256, 0, st>>>(q, k, v, o, dout, lse, pb, dq, dd);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   dim3 g2((pb.max_seqlen + kRowsPerBlock - 1) / kRowsPerBlock, pb.hkv, pb.batch);
+  LaunchScope scope(K_BWD_FP32_DKDV, st);
   bwd_fp32_dkdv_kernel<D><<<g2, 256, 0, st>>>(q, k, v, dout, lse, dd, pb, dk, dv);
   return cudaGetLastError();
 }

@@ -366,6 +366,7 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   if (e != cudaSuccess) return e;
   const int pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
   dim3 grid(pb.hq, pb.batch, pairs);
+  LaunchScope scope(K_FWD_BF16, stream);
   fwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -37,6 +37,27 @@ cudaError_t launch_bwd_fp32(const Problem& pb, const float* q, const float* k, c
                             const float* dout, const float* lse, float* dq, float* dk, float* dv, void* workspace,
                             cudaStream_t stream);
 
+// Launch bookkeeping: every kernel launch is wrapped in a LaunchScope, which counts it
+// and, while timing is enabled, brackets it with CUDA events on its stream.
+enum KernelKind : int {
+  K_FWD_BF16 = 0,
+  K_BWD_PREPROCESS,
+  K_BWD_BF16,
+  K_BWD_DQ_CONVERT,
+  K_FWD_FP32,
+  K_BWD_FP32_DQ,
+  K_BWD_FP32_DKDV,
+  K_NUM_KINDS
+};
+const char* kernel_kind_name(int kind);
+struct LaunchScope {
+  LaunchScope(int kind, cudaStream_t stream);
+  ~LaunchScope();
+  int kind;
+  cudaStream_t stream;
+  int slot;   // event pair index, -1 when timing is off
+};
+
 // Host helper shared by the launchers: encodes a 3-D bf16 TMA descriptor over a
 // [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that
 // matches a box_inner * 2-byte row (128 B or 64 B).
