@@ -102,6 +102,27 @@ attn_status attn_bwd(const void *q, const void *k, const void *v,
                      void *dq, void *dk, void *dv,
                      void *workspace, size_t workspace_bytes, void *stream);
 
+/* Backward without a caller-provided workspace.  (The pages describe no counterpart; this
+ * exists for callers that cannot allocate device memory where they run the backward:
+ * engines that reserve all device memory up front and forbid allocation later, and plain
+ * C hosts with no allocator to take a workspace from.)  Same arguments, layouts and
+ * results as attn_bwd, minus the workspace: the scratch comes from a 64 MiB array in the
+ * library's device globals, held on every GPU that uses the library until the process
+ * exits.  A problem whose attn_bwd_workspace_size() exceeds 64 MiB is rejected with
+ * ATTN_ERR_INVALID_ARG (attn_last_error_message() says how much it needs); nothing is ever
+ * allocated.  The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.  Every call
+ * shares the one array, and the backward clears the parts that must start at zero on
+ * every call; calls whose GPU work overlaps (other streams, other host threads on the
+ * same device) race on it and must not be made. */
+attn_status attn_bwd_noalloc(const void *q, const void *k, const void *v,
+                             const void *o, const void *dout, const float *lse,
+                             const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
+                             int32_t max_seqlen, int32_t total_tokens,
+                             int32_t hq, int32_t hkv, int32_t d,
+                             float scale, int32_t causal, int32_t dtype,
+                             void *dq, void *dk, void *dv, void *stream);
+
 /* Workspace bytes attn_fwd / attn_bwd need for these shape arguments (0 = none). */
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,
                                int32_t hq, int32_t hkv, int32_t d, int32_t dtype);

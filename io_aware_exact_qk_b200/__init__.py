@@ -68,6 +68,9 @@ def load_library():
     lib.attn_profile_kernel_name.restype = ctypes.c_char_p
     lib.attn_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), i32]
     lib.attn_profile_collect.restype = ctypes.c_int
+    lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                     vp, vp, vp, vp]
+    lib.attn_bwd_noalloc.restype = ctypes.c_int
     lib.attn_launch_count.argtypes = []
     lib.attn_launch_count.restype = ctypes.c_int64
     _lib = lib
@@ -158,6 +161,26 @@ def attn_bwd(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scale=None, 
     _check(lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(cu_seqlens), b, seqlen,
                         ms, T, hq, hkv, d, float(scale), int(bool(causal)), _dtype_code(q), _ptr(dq), _ptr(dk),
                         _ptr(dv), _ptr(workspace), ws if workspace is not None else 0, _stream(stream)))
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scale=None, causal=False,
+                     batch=None, dq=None, dk=None, dv=None, stream=None):
+    """Backward for callers that cannot allocate device memory when they run it (engines
+    that reserve all device memory up front, hosts with no allocator to give a
+    workspace from).  Same results as attn_bwd; the scratch is the library's built-in
+    64 MiB array, so larger problems are refused and concurrent calls on one device race.
+    (dq/dk/dv are allocated here only when not passed in.)"""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(cu_seqlens), b,
+                                seqlen, ms, T, hq, hkv, d, float(scale), int(bool(causal)), _dtype_code(q),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))
     return dq, dk, dv
 
 

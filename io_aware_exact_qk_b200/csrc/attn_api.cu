@@ -115,6 +115,14 @@ std::atomic<int64_t> g_launches{0};
 
 }  // namespace
 
+int record_error(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return status;
+}
+
 const char* kernel_kind_name(int kind) {
   static const char* names[K_NUM_KINDS] = {"fwd_bf16_sm100",  "bwd_preprocess",       "bwd_bf16_sm100",
                                            "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",

@@ -58,6 +58,10 @@ struct LaunchScope {
   int slot;   // event pair index, -1 when timing is off
 };
 
+// Records `fmt` as the calling thread's last error message (attn_last_error_message) and
+// returns `status`.
+int record_error(int status, const char* fmt, ...);
+
 // Host helper shared by the launchers: encodes a 3-D bf16 TMA descriptor over a
 // [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that
 // matches a box_inner * 2-byte row (128 B or 64 B).
