@@ -40,8 +40,9 @@
 // + dK (128) + two dQ^T buffers (2 x 64) = 512 columns.  d <= 64 uses BM = 128 and
 // dQ_i = dS K_j (M = 128 query rows, N = d): 128 + 128 + 4 d <= 512 columns.
 //
-// Warp roles (320 threads): warps 0-3 compute (P^T, dS^T, epilogue of dK/dV), warps 4-7
-// dQ drain, warp 8 TMA producer (+ LSE / D rows into SMEM), warp 9 MMA issuer.
+// Warp roles (448 threads): two compute warpgroups, each owning half of the query columns
+// of every step (P^T, dS^T) and one of the dK / dV epilogues; a dQ drain warpgroup; a TMA
+// producer warp (+ LSE / D rows into SMEM, one step ahead); an MMA issuer warp.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -50,13 +51,15 @@ namespace attn {
 namespace {
 
 constexpr int kKeys = 128;   // keys per CTA == TMEM lanes
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct BwdCfg {
   static constexpr bool DQT = (D == 128);          // dQ^T form (see file comment)
+  static constexpr int STAGES = DQT ? 3 : 2;      // Q_i / dO_i / LSE_i / D_i ring depth
   static constexpr int BM = DQT ? 64 : 128;       // query rows per step
+  static constexpr int HALF = BM / 2;             // query columns per compute warpgroup
   static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span of Q/K/V/dO rows (bytes)
   static constexpr int PANEL = SW / 2;
   static constexpr int NPANEL = D / PANEL;
@@ -79,25 +82,32 @@ struct BwdCfg {
   // shared memory map (offsets from the 1024-aligned base)
   static constexpr int O_K = 0;
   static constexpr int O_V = O_K + KV_TILE_BYTES;
-  static constexpr int O_Q = O_V + KV_TILE_BYTES;          // 2 stages
-  static constexpr int O_DO = O_Q + 2 * Q_TILE_BYTES;      // 2 stages
-  static constexpr int O_DS = O_DO + 2 * Q_TILE_BYTES;     // 2 buffers
-  static constexpr int O_LSE = O_DS + 2 * DS_BYTES;        // 2 stages x BM floats (LSE * log2 e)
-  static constexpr int O_DD = O_LSE + 2 * BM * 4;          // 2 stages x BM floats (D)
-  static constexpr int O_BAR = O_DD + 2 * BM * 4;
+  static constexpr int O_Q = O_V + KV_TILE_BYTES;              // STAGES
+  static constexpr int O_DO = O_Q + STAGES * Q_TILE_BYTES;      // STAGES
+  static constexpr int O_DS = O_DO + STAGES * Q_TILE_BYTES;     // 2 buffers
+  static constexpr int O_LSE = O_DS + 2 * DS_BYTES;            // STAGES x BM floats (LSE * log2 e)
+  static constexpr int O_DD = O_LSE + STAGES * BM * 4;         // STAGES x BM floats (D)
+  // dQ staging tile for the bulk reduction, [BM query rows][d] fp32.  d = 128: plain
+  // row-major (written column-wise, one feature per thread).  d <= 64: 32-float panels
+  // with the 128-byte swizzle (written row-wise, one query row per thread).
+  static constexpr int STG_ALIGN = DQT ? 128 : 1024;            // swizzled tiles need 1024
+  static constexpr int O_STG = (O_DD + STAGES * BM * 4 + STG_ALIGN - 1) & ~(STG_ALIGN - 1);
+  static constexpr int STG_PANEL_BYTES = BM * 128;              // d <= 64: [BM rows][32 floats]
+  static constexpr int STG_BYTES = BM * D * 4;
+  static constexpr int O_BAR = O_STG + STG_BYTES;
   // barriers
   static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;     // 2
-  static constexpr int B_QEMPTY = 3;    // 2
-  static constexpr int B_ST = 5;
-  static constexpr int B_DPT = 6;
-  static constexpr int B_PT = 7;
-  static constexpr int B_DS = 8;
-  static constexpr int B_DSFREE = 9;    // 2
-  static constexpr int B_DQFULL = 11;   // 2
-  static constexpr int B_DQEMPTY = 13;  // 2
-  static constexpr int B_DONE = 15;
-  static constexpr int NBARS = 16;
+  static constexpr int B_QFULL = 1;                  // STAGES
+  static constexpr int B_QEMPTY = B_QFULL + STAGES;  // STAGES
+  static constexpr int B_ST = B_QEMPTY + STAGES;
+  static constexpr int B_DPT = B_ST + 1;
+  static constexpr int B_PT = B_DPT + 1;
+  static constexpr int B_DS = B_PT + 1;
+  static constexpr int B_DSFREE = B_DS + 1;          // 2
+  static constexpr int B_DQFULL = B_DSFREE + 2;      // 2
+  static constexpr int B_DQEMPTY = B_DQFULL + 2;     // 2
+  static constexpr int B_DONE = B_DQEMPTY + 2;
+  static constexpr int NBARS = B_DONE + 1;
   static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 16;
 };
 
@@ -128,13 +138,20 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Warp roles (448 threads):
+//   warps 0-3   compute, query columns [0, BM/2) of every step, then the dV epilogue
+//   warps 4-7   compute, query columns [BM/2, BM), then the dK epilogue
+//   warps 8-11  dQ drain
+//   warp  12    producer (TMA for K, V, Q_i, dO_i; LSE_i, D_i rows into SMEM)
+//   warp  13    MMA issuer
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int BM = C::BM;
+  constexpr int HALF = C::HALF;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -148,9 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = blockIdx.x;        // kv head
-  const int b = blockIdx.y;        // sequence
-  const int jt = blockIdx.z;       // key tile (0 = most query tiles under causal: first)
+  const int jt = blockIdx.x;       // key tile: the tiles of one head run together (L2 reuse)
+  const int g = blockIdx.y;        // kv head
+  const int b = blockIdx.z;        // sequence
   const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
   const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
   const int kv0 = jt * kKeys;
@@ -165,8 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
-      if (i == C::B_QFULL || i == C::B_QFULL + 1) cnt = 32;
-      if (i == C::B_PT || i == C::B_DS || i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 128;
+      if (i >= C::B_QFULL && i < C::B_QFULL + C::STAGES) cnt = 32;
+      if (i == C::B_PT || i == C::B_DS) cnt = 256;
+      if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 128;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -176,18 +194,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQ);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ---------------- producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per step ----------
     if (lane == 0) {
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE_BYTES);
@@ -196,19 +215,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + C::O_V + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
       }
     }
+    // LSE_i * log2(e) and D_i of the next step are loaded into registers one step ahead,
+    // so their global-memory latency overlaps the wait for a free stage.  Query rows past
+    // the sequence get LSE = +inf (P = 0 there without a mask) and D = 0.
+    constexpr int PER_LANE = BM / 32;
+    float nl[PER_LANE], nd[PER_LANE];
+    auto fetch = [&](int n) {
+      int h, i;
+      it.head_tile(n, g, &h, &i);
+#pragma unroll
+      for (int e = 0; e < PER_LANE; ++e) {
+        const int qi = i * BM + e * 32 + lane;
+        const bool ok = qi < len;
+        const size_t idx = (size_t)h * p.total_tokens + seq_start + (ok ? qi : 0);
+        nl[e] = ok ? p.lse[idx] * kLog2e : INFINITY;
+        nd[e] = ok ? p.dd[idx] : 0.f;
+      }
+    };
+    fetch(0);
     for (int n = 0; n < n_steps; ++n) {
-      const int s = n & 1;
-      if (!mbar_wait(bar(C::B_QEMPTY + s), ((n >> 1) & 1) ^ 1, abort_flag)) break;
+      const int s = n % C::STAGES;
+      if (!mbar_wait(bar(C::B_QEMPTY + s), ((n / C::STAGES) & 1) ^ 1, abort_flag)) break;
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
-      for (int c = lane; c < BM; c += 32) {
-        const int qi = q0 + c;
-        const bool ok = qi < len;
-        const size_t idx = (size_t)h * p.total_tokens + seq_start + qi;
-        s_lse[s * BM + c] = ok ? p.lse[idx] * kLog2e : 0.f;
-        s_dd[s * BM + c] = ok ? p.dd[idx] : 0.f;
+#pragma unroll
+      for (int e = 0; e < PER_LANE; ++e) {
+        s_lse[s * BM + e * 32 + lane] = nl[e];
+        s_dd[s * BM + e * 32 + lane] = nd[e];
       }
+      if (n + 1 < n_steps) fetch(n + 1);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
         for (int pn = 0; pn < C::NPANEL; ++pn) {
@@ -221,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(C::B_QFULL + s));
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t id_sdp = idesc_bf16_f32(kKeys, BM, false, false);   // K Q^T, V dO^T
@@ -240,12 +276,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + d_col, a, bd, id_sdp, kk > 0 ? 1u : 0u);
         }
       };
-      // D[128 keys x d] += A^T(TMEM, bf16 over BM queries) * Y_i (BM x d, MN-major)
+      // D[128 keys x d] += A^T(TMEM, bf16 over BM queries) * Y_i (BM x d, MN-major).
+      // Each compute warpgroup packs its half of the queries into the first columns of
+      // its own half of the fp32 region, so queries [h*HALF, (h+1)*HALF) sit at columns
+      // h*HALF + (q - h*HALF)/2.
       auto issue_grad = [&](uint32_t a_col, uint32_t y_off, uint32_t d_col, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
+          const int qb = kk * 16;
+          const int hh = qb / HALF;
+          const uint32_t col = a_col + hh * HALF + (qb - hh * HALF) / 2;
           const uint64_t bd = smem_desc(sbase + y_off + kk * 16 * C::SW, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
-          mma_ts(tmem + d_col, tmem + a_col + kk * 8, bd, id_grad, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + d_col, tmem + col, bd, id_grad, (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto issue_dq = [&](int dsbuf, uint32_t d_col) {
@@ -269,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(C::B_DPT));
       }
       for (int n = 0; ok && n < n_steps; ++n) {
-        const int s = n & 1;
+        const int s = n % C::STAGES;
+        const int s1 = (n + 1) % C::STAGES;
+        const int b2 = n & 1;
         const uint32_t q_off = C::O_Q + s * C::Q_TILE_BYTES;
         const uint32_t do_off = C::O_DO + s * C::Q_TILE_BYTES;
         const bool more = n + 1 < n_steps;
@@ -277,97 +321,111 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_grad(C::T_ST, do_off, C::T_DV, n > 0);                  // dV += P^T dO
         if (more) {
-          if (!mbar_wait(bar(C::B_QFULL + (s ^ 1)), ((n + 1) >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(bar(C::B_QFULL + s1), ((n + 1) / C::STAGES) & 1, abort_flag)) break;
           tc_fence_after();
-          issue_sdp(C::O_K, C::O_Q + (s ^ 1) * C::Q_TILE_BYTES, C::T_ST);   // S^T for the next step
+          issue_sdp(C::O_K, C::O_Q + s1 * C::Q_TILE_BYTES, C::T_ST);   // S^T for the next step
           mma_commit(bar(C::B_ST));
         }
         if (!mbar_wait(bar(C::B_DS), n & 1, abort_flag)) break;
         tc_fence_after();
         issue_grad(C::T_DPT, q_off, C::T_DK, n > 0);                  // dK += dS^T Q
         mma_commit(bar(C::B_QEMPTY + s));
-        if (!mbar_wait(bar(C::B_DQEMPTY + s), ((n >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar(C::B_DQEMPTY + b2), ((n >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        issue_dq(s, C::T_DQ + s * C::DQ_COLS);                         // dQ_i partial
-        mma_commit(bar(C::B_DQFULL + s));
-        mma_commit(bar(C::B_DSFREE + s));
+        issue_dq(b2, C::T_DQ + b2 * C::DQ_COLS);                       // dQ_i partial
+        mma_commit(bar(C::B_DQFULL + b2));
+        mma_commit(bar(C::B_DSFREE + b2));
         if (more) {
-          issue_sdp(C::O_V, C::O_DO + (s ^ 1) * C::Q_TILE_BYTES, C::T_DPT);  // dP^T for the next step
+          issue_sdp(C::O_V, C::O_DO + s1 * C::Q_TILE_BYTES, C::T_DPT);  // dP^T for the next step
           mma_commit(bar(C::B_DPT));
         }
       }
       mma_commit(bar(C::B_DONE));
     }
-  } else if (warp < 4) {
-    // ---------------- compute: P^T, dS^T (one key row per thread) ----------------
-    const int lane_base = warp * 32;
+  } else if (warp < 8) {
+    // ---------------- compute: P^T, dS^T for one key row and half of the query columns ----
+    const int half = warp >> 2;                   // 0: columns [0, HALF), 1: [HALF, BM)
+    const int lane_base = (warp & 3) * 32;
     const int kr = lane_base + lane;              // key row inside the tile
     const int kj = kv0 + kr;                      // key index inside the sequence
+    const int c0 = half * HALF;                   // first query column of this thread
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int n = 0; n < n_steps; ++n) {
-      const int s = n & 1;
+      const int s = n % C::STAGES;
+      const int b2 = n & 1;
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
-      // visible query columns c: q0 + c < len, and (causal) q0 + c >= kj; key inside the sequence
-      int c_lo = 0, c_hi = BM;                    // [c_lo, c_hi)
-      if (q0 + BM > len) c_hi = len - q0;
-      if (p.causal && kj - q0 > c_lo) c_lo = kj - q0;
-      if (kj >= len) c_hi = 0;
-      if (!mbar_wait(bar(C::B_QFULL + s), (n >> 1) & 1, abort_flag)) { ok = false; break; }
+      // Columns c < c_lo are hidden by the causal mask; a key past the sequence hides all.
+      // (Query rows past the sequence carry LSE = +inf, so they come out as P = 0.)
+      int c_lo = p.causal ? kj - q0 : 0;
+      if (kj >= len) c_lo = BM;
+      const bool masked = c_lo > c0;
+      if (!mbar_wait(bar(C::B_QFULL + s), (n / C::STAGES) & 1, abort_flag)) { ok = false; break; }
       if (!mbar_wait(bar(C::B_ST), n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const float* lse = s_lse + s * BM;
-      const float* dd = s_dd + s * BM;
-      float pr[BM];
+      const float4* lse4 = reinterpret_cast<const float4*>(s_lse + s * BM + c0);
+      const float4* dd4 = reinterpret_cast<const float4*>(s_dd + s * BM + c0);
+      float pr[HALF];
 #pragma unroll
-      for (int cb = 0; cb < BM; cb += 32) {
+      for (int cb = 0; cb < HALF; cb += 32) {
         uint32_t r[32];
-        tmem_ld32(trow + C::T_ST + cb, r);
+        tmem_ld32(trow + C::T_ST + c0 + cb, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = cb + e;
-          const float x = fmaf(__uint_as_float(r[e]), sl2, -lse[c]);
-          pr[c] = (c >= c_lo && c < c_hi) ? ex2(x) : 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l4 = lse4[(cb >> 2) + e4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = e4 * 4 + u;
+            pr[cb + e] = ex2(fmaf(__uint_as_float(r[e]), sl2, -lv[u]));
+          }
         }
       }
+      if (masked) {
 #pragma unroll
-      for (int cb = 0; cb < BM; cb += 32) {
+        for (int c = 0; c < HALF; ++c)
+          if (c0 + c < c_lo) pr[c] = 0.f;
+      }
+#pragma unroll
+      for (int cb = 0; cb < HALF; cb += 32) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(pr[cb + 2 * e], pr[cb + 2 * e + 1]);
-        tmem_st16(trow + C::T_ST + cb / 2, w);
+        tmem_st16(trow + C::T_ST + c0 + cb / 2, w);   // inside this warpgroup's own columns
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::B_PT));
       // dS^T = P^T o (dP^T - D): to TMEM (over dP^T) and to the swizzled SMEM buffer
-      if (!mbar_wait(bar(C::B_DSFREE + s), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_DSFREE + b2), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       if (!mbar_wait(bar(C::B_DPT), n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint8_t* ds_smem = smem + C::O_DS + s * C::DS_BYTES;
+      uint8_t* ds_smem = smem + C::O_DS + b2 * C::DS_BYTES;
 #pragma unroll
-      for (int cb = 0; cb < BM; cb += 32) {
+      for (int cb = 0; cb < HALF; cb += 32) {
         uint32_t r[32];
-        tmem_ld32(trow + C::T_DPT + cb, r);
+        tmem_ld32(trow + C::T_DPT + c0 + cb, r);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = cb + 2 * e;
-          const float d0 = pr[c] * (__uint_as_float(r[2 * e]) - dd[c]);
-          const float d1 = pr[c + 1] * (__uint_as_float(r[2 * e + 1]) - dd[c + 1]);
-          w[e] = pack_bf16x2(d0, d1);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 d4 = dd4[(cb >> 2) + e4];
+          const int e = e4 * 4;
+          w[2 * e4] = pack_bf16x2(pr[cb + e] * (__uint_as_float(r[e]) - d4.x),
+                                  pr[cb + e + 1] * (__uint_as_float(r[e + 1]) - d4.y));
+          w[2 * e4 + 1] = pack_bf16x2(pr[cb + e + 2] * (__uint_as_float(r[e + 2]) - d4.z),
+                                      pr[cb + e + 3] * (__uint_as_float(r[e + 3]) - d4.w));
         }
-        tmem_st16(trow + C::T_DPT + cb / 2, w);
-        // queries cb..cb+31 live in panel cb/64, 16-byte chunks (cb%64)/8 .. +3
-        uint8_t* panel = ds_smem + (cb / 64) * C::DS_PANEL_BYTES;
+        tmem_st16(trow + C::T_DPT + c0 + cb / 2, w);
+        // queries c0+cb .. +31 live in panel (c0+cb)/64, 16-byte chunks ((c0+cb)%64)/8 .. +3
+        uint8_t* panel = ds_smem + ((c0 + cb) / 64) * C::DS_PANEL_BYTES;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = (cb % 64) / 8 + ch;
+          const int chunk = ((c0 + cb) % 64) / 8 + ch;
           *reinterpret_cast<uint4*>(panel + sw128_offset(kr, chunk)) =
               make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
         }
@@ -377,74 +435,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::B_DS));
     }
-    // ---------------- epilogue: dK = scale * acc, dV ----------------
+    // ---------------- epilogue: warps 0-3 write dV, warps 4-7 write dK = scale * acc ------
     if (ok && mbar_wait(bar(C::B_DONE), 0, abort_flag)) {
       tc_fence_after();
       const bool row_ok = kj < len;
       const size_t orow = ((size_t)(seq_start + kj) * p.hkv + g) * D;
+      __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + orow;
+      const float mul = half == 0 ? 1.f : p.scale;
+      const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
-        const float mul = which == 0 ? 1.f : p.scale;
-        const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + col + cb, r);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint32_t w[16];
 #pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t r[32];
-          tmem_ld32(trow + col + cb, r);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint32_t w[16];
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+          uint4* o4 = reinterpret_cast<uint4*>(dst + cb);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
-            uint4* o4 = reinterpret_cast<uint4*>(dst + cb);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-          }
+          for (int e = 0; e < 4; ++e) o4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ---------------- dQ drain: TMEM partial -> fp32 atomics into the accumulator ---------
     const int lane_base = (warp & 3) * 32;
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     for (int n = 0; n < n_steps; ++n) {
-      const int s = n & 1;
+      const int b2 = n & 1;
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
-      if (!mbar_wait(bar(C::B_DQFULL + s), (n >> 1) & 1, abort_flag)) break;
+      if (!mbar_wait(bar(C::B_DQFULL + b2), (n >> 1) & 1, abort_flag)) break;
       tc_fence_after();
       uint32_t r[C::DQ_COLS / 32][32];
 #pragma unroll
-      for (int cb = 0; cb < C::DQ_COLS / 32; ++cb) tmem_ld32(trow + C::T_DQ + s * C::DQ_COLS + cb * 32, r[cb]);
+      for (int cb = 0; cb < C::DQ_COLS / 32; ++cb) tmem_ld32(trow + C::T_DQ + b2 * C::DQ_COLS + cb * 32, r[cb]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DQEMPTY + s));
+      mbar_arrive(bar(C::B_DQEMPTY + b2));
       if (C::DQT) {
-        // lane = feature c, registers = the BM query rows of this step
+        // lane = feature c, registers = the BM query rows of this step.  The partial is
+        // transposed into a [BM][d] fp32 staging tile and added into the accumulator by
+        // one bulk tensor reduction (query rows past the sequence carry exact zeros).
         const int c = lane_base + lane;
-        float* base = p.dq_acc + ((size_t)(seq_start + q0) * p.hq + h) * D + c;
-        const int rows = min(BM, len - q0);
+        if (warp == 8 && lane == 0) bulk_wait_group_read0();   // previous reduce has read the tile
+        named_barrier_sync(1, 128);
+        float* stg = reinterpret_cast<float*>(smem + C::O_STG);
 #pragma unroll
-        for (int e = 0; e < BM; ++e)
-          if (e < rows) atomicAdd(base + (size_t)e * p.hq * D, __uint_as_float(r[e / 32][e % 32]));
+        for (int e = 0; e < BM; ++e) stg[e * D + c] = __uint_as_float(r[e / 32][e % 32]);
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (warp == 8 && lane == 0) {
+          tma_reduce_add_3d(&tmDQ, sbase + C::O_STG, 0, h, seq_start + q0);
+          bulk_commit_group();
+        }
       } else {
-        // lane = query row, registers = its d features (contiguous in memory)
-        const int qr = q0 + lane_base + lane;
-        if (qr < len) {
-          float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)(seq_start + qr) * p.hq + h) * D);
+        // lane = query row, registers = its d features.  Each 32-feature panel row is 128
+        // bytes, stored with the 128-byte swizzle (16-byte chunk j of row q at j ^ (q & 7))
+        // so that eight consecutive rows hit eight different bank groups; the tensor map
+        // uses the same swizzle for the bulk reduction.
+        const int qr = lane_base + lane;
+        if (warp == 8 && lane == 0) bulk_wait_group_read0();
+        named_barrier_sync(1, 128);
+        uint8_t* stg = smem + C::O_STG;
 #pragma unroll
-          for (int e = 0; e < D / 4; ++e)
-            atomicAdd(dst + e, make_float4(__uint_as_float(r[(4 * e) / 32][(4 * e) % 32]),
-                                           __uint_as_float(r[(4 * e + 1) / 32][(4 * e + 1) % 32]),
-                                           __uint_as_float(r[(4 * e + 2) / 32][(4 * e + 2) % 32]),
-                                           __uint_as_float(r[(4 * e + 3) / 32][(4 * e + 3) % 32])));
+        for (int pn = 0; pn < D / 32; ++pn)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int e = pn * 32 + j * 4;
+            *reinterpret_cast<uint4*>(stg + pn * C::STG_PANEL_BYTES + sw128_offset(qr, j)) =
+                make_uint4(r[e / 32][e % 32], r[e / 32][e % 32 + 1], r[e / 32][e % 32 + 2], r[e / 32][e % 32 + 3]);
+          }
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (warp == 8 && lane == 0) {
+          for (int pn = 0; pn < D / 32; ++pn)
+            tma_reduce_add_3d(&tmDQ, sbase + C::O_STG + pn * C::STG_PANEL_BYTES, pn * 32, h, seq_start + q0);
+          bulk_commit_group();
         }
       }
     }
   }
 
+  if (warp == 8 && lane == 0) bulk_wait_group0();   // bulk reductions complete
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -541,8 +617,9 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  alignas(64) CUtensorMap tq, tk, tv, tdo;
-  if (!encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
+  alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!encode_tma_3d_f32(&tdq, dq_acc, D, pb.hq, pb.total_tokens, C::DQT ? D : 32, C::BM) ||
+      !encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
       !encode_tma_3d(&tdo, dout, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
       !encode_tma_3d(&tk, k, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys) ||
       !encode_tma_3d(&tv, v, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys))
@@ -564,10 +641,10 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   p.dv = static_cast<__nv_bfloat16*>(dv);
   cudaError_t e = cudaFuncSetAttribute(bwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(pb.hkv, pb.batch, (pb.max_seqlen + kKeys - 1) / kKeys);
+  dim3 grid((pb.max_seqlen + kKeys - 1) / kKeys, pb.hkv, pb.batch);
   {
     LaunchScope scope(K_BWD_BF16, stream);
-    bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;

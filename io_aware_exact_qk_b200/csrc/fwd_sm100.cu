@@ -96,13 +96,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
-  const int pair = gridDim.z - 1 - blockIdx.z;   // heaviest (last) query tiles first
+  // Launch order.  Without a mask every CTA does the same work, and the query-tile pairs
+  // of one head are adjacent (grid x) so their shared K/V stream is served from L2.  With
+  // the causal mask the work grows with the pair index, so the heaviest pairs of every
+  // head go first (grid z, reversed) to keep the tail of the launch short.
+  int pair, h, b;
+  if (p.causal) {
+    h = blockIdx.x;
+    b = blockIdx.y;
+    pair = gridDim.z - 1 - blockIdx.z;
+  } else {
+    pair = blockIdx.x;
+    h = blockIdx.y;
+    b = blockIdx.z;
+  }
   const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
   const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
   if (len > p.max_seqlen) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) report_error(ATTN_DEVERR_SEQLEN);
+    if (threadIdx.x == 0 && pair == 0 && h == 0) report_error(ATTN_DEVERR_SEQLEN);
   }
   const int q0 = pair * 2 * kRows;
   if (q0 >= len) return;   // uniform over the CTA, before any barrier or TMEM use
@@ -365,7 +376,7 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
-  dim3 grid(pb.hq, pb.batch, pairs);
+  const dim3 grid = pb.causal ? dim3(pb.hq, pb.batch, pairs) : dim3(pairs, pb.hq, pb.batch);
   LaunchScope scope(K_FWD_BF16, stream);
   fwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

@@ -66,5 +66,8 @@ int record_error(int status, const char* fmt, ...);
 // [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that
 // matches a box_inner * 2-byte row (128 B or 64 B).
 bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows);
+// The same over an fp32 [rows, heads, d] tensor; a 32-float (128-byte) box row uses the
+// 128-byte swizzle, any other width is unswizzled.  Used for bulk reductions.
+bool encode_tma_3d_f32(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows);
 
 }  // namespace attn
