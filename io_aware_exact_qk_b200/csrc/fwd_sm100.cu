@@ -41,7 +41,6 @@ constexpr int kRows = 128;                 // query rows per tile == TMEM lanes
 constexpr int kKeys = 128;                 // keys per K/V tile
 constexpr float kRescaleSkip = 8.0f;       // log2 units, see file comment
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kThreads = 320;
 
 template <int D>
@@ -72,7 +71,8 @@ struct FwdCfg {
 struct FwdParams {
   const int32_t* cu_seqlens;
   int32_t seqlen, max_seqlen, total_tokens, hq, hkv;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e), rounded to fp32
+  double lse_skew;   // scale_log2 * ln 2 - scale, in double: the rounding of scale_log2
   int32_t causal;
   __nv_bfloat16* o;
   float* lse;
@@ -239,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + 2 * kKeys + t * D;
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY;   // running max in log2 units (possibly stale by < 8)
+    float mx_used = 0.f;        // the raw score maximum that m_used was formed from
     float l = 0.f;              // running sum of exp2(x - m_used)
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
@@ -275,7 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
       const float m_cand = mx * sl2;
       float m_new = m_used;
-      if (m_cand > m_used + kRescaleSkip) m_new = m_cand;
+      if (m_cand > m_used + kRescaleSkip) {
+        m_new = m_cand;
+        mx_used = mx;
+      }
       const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
       float rowsum = 0.f;
       uint32_t pk[64];
@@ -339,7 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (row_ok) {
-        const float lse = l > 0.f ? (m_used == -INFINITY ? 0.f : m_used) * kLn2 + logf(l) : -INFINITY;
+        // LSE = m ln 2 + ln l, evaluated in double from the exact fp32 values the
+        // exponentials used (m_used, l), minus the first-order effect of scale_log2 being
+        // rounded to fp32 (exact when one score dominates the row), then rounded once.
+        float lse = -INFINITY;
+        if (l > 0.f)
+          lse = (float)((double)m_used * 0.6931471805599453 + log((double)l) - p.lse_skew * (double)mx_used);
         p.lse[(size_t)h * p.total_tokens + seq_start + qi] = lse;
       }
     }
@@ -370,6 +379,7 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   p.hq = pb.hq;
   p.hkv = pb.hkv;
   p.scale_log2 = pb.scale * kLog2e;
+  p.lse_skew = (double)p.scale_log2 * 0.6931471805599453 - (double)pb.scale;
   p.causal = pb.causal;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;

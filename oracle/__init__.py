@@ -37,6 +37,9 @@ def _bind(lib):
     lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, ip, i32, i32, i32, i32, f64, i32,
                                     up, up, dp, dp, dp, dp, dp, i32]
     lib.oracle_attn_bwd.restype = ctypes.c_int
+    lib.oracle_attn_bwd_ex.argtypes = [dp, dp, dp, dp, ip, i32, i32, i32, i32, f64, i32,
+                                       up, up, dp, dp, dp, dp, dp, dp, dp, i32]
+    lib.oracle_attn_bwd_ex.restype = ctypes.c_int
     lib.oracle_attn_probs.argtypes = [dp, dp, i32, i32, f64, i32, dp, dp]
     lib.oracle_attn_probs.restype = ctypes.c_int
     _lib = lib
@@ -115,10 +118,12 @@ def attn_fwd(q, k, v, cu_seqlens=None, scale=None, causal=False, rows=None, thre
 
 
 def attn_bwd(q, k, v, do, cu_seqlens=None, scale=None, causal=False, rows=None, keys=None,
-             threads=None):
+             threads=None, o=None, lse=None):
     """dQ [T,Hq,d], dK, dV [T,Hkv,d], and the oracle's own O, LSE (float64).
     ``rows`` / ``keys`` (optional token indices) limit which dQ rows / dK,dV keys are
-    produced; the others are NaN."""
+    produced; the others are NaN.  ``o`` [T,Hq,d] / ``lse`` [Hq,T] (optional) are the
+    forward's saved outputs: D is then formed from ``o`` and P from ``lse`` (the backward
+    as a function of its inputs); without them the result is the exact gradient."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     T, hq, d = q.shape
     hkv = k.shape[1]
@@ -128,17 +133,20 @@ def attn_bwd(q, k, v, do, cu_seqlens=None, scale=None, causal=False, rows=None, 
     dq = np.full((T, hq, d), np.nan)
     dk = np.full((T, hkv, d), np.nan)
     dv = np.full((T, hkv, d), np.nan)
-    o = np.empty((T, hq, d))
-    lse = np.empty((hq, T))
     rsel, ksel = _sel(rows, T), _sel(keys, T)
-    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu, ctypes.c_int32),
-                                 len(cu) - 1, hq, hkv, d, float(scale), int(bool(causal)),
-                                 _ptr(rsel, ctypes.c_uint8), _ptr(ksel, ctypes.c_uint8),
-                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(o), _ptr(lse),
-                                 threads or default_threads())
+    o_in = None if o is None else _f64(o)
+    lse_in = None if lse is None else _f64(lse)
+    o_out = np.empty((T, hq, d))
+    lse_out = np.empty((hq, T))
+    rc = _load().oracle_attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu, ctypes.c_int32),
+                                    len(cu) - 1, hq, hkv, d, float(scale), int(bool(causal)),
+                                    _ptr(rsel, ctypes.c_uint8), _ptr(ksel, ctypes.c_uint8),
+                                    _ptr(o_in), _ptr(lse_in),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(o_out), _ptr(lse_out),
+                                    threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
-    return dq, dk, dv, o, lse
+    return dq, dk, dv, o_out, lse_out
 
 
 def attn_probs(q, k, scale=None, causal=False):

@@ -345,13 +345,21 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v,
 /* Backward: dq [T,hq,d], dk/dv [T,hkv,d].  The oracle forms its own O, LSE and D from
  * the definition first (all rows of every head).  row_sel / key_sel (optional, [T])
  * restrict which dQ rows and which dK/dV keys are produced; others stay untouched.
- * o_out / lse_out (optional) receive the forward results. */
-int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
-                    const int32_t *cu_seqlens, int32_t nseq,
-                    int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
-                    const uint8_t *row_sel, const uint8_t *key_sel,
-                    double *dq, double *dk, double *dv,
-                    double *o_out, double *lse_out, int32_t nthreads)
+ * o_out / lse_out (optional) receive the forward results.
+ *
+ * o_in / lse_in (optional) make this the backward *as a function of its inputs*: the
+ * backward takes the forward's saved O and statistics ("前向: 只保存输出 O 与每块的
+ * softmax 统计量"; "反向重算流程": recompute S and P from Q/K/V and those statistics).
+ * When o_in is given, D_i = sum_c dO_ic o_in_ic; when lse_in is given,
+ * P_ij = exp(S_ij - lse_in_i).  Without them the oracle's own O and LSE are used, which
+ * is the exact gradient of the forward definition. */
+int oracle_attn_bwd_ex(const double *q, const double *k, const double *v, const double *dout,
+                       const int32_t *cu_seqlens, int32_t nseq,
+                       int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                       const uint8_t *row_sel, const uint8_t *key_sel,
+                       const double *o_in, const double *lse_in,
+                       double *dq, double *dk, double *dv,
+                       double *o_out, double *lse_out, int32_t nthreads)
 {
     int rc = check_args(cu_seqlens, nseq, hq, hkv, d);
     if (rc) return rc;
@@ -372,12 +380,37 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
     P.o = o; P.lse = lse; P.dd = dd;
     P.dq = dq; P.dk = dk; P.dv = dv;
     rc = run_items(&P, 0, hq, nthreads);          /* O, LSE, D for every row */
+    if (!rc && (o_in || lse_in)) {                 /* the given O / LSE replace the oracle's */
+        for (int64_t t = 0; t < T; ++t)
+            for (int h = 0; h < hq; ++h) {
+                if (lse_in) lse[(int64_t)h * T + t] = lse_in[(int64_t)h * T + t];
+                if (o_in) {
+                    const double *og = o_in + (t * hq + h) * d;
+                    const double *dog = dout + (t * hq + h) * d;
+                    double dsum = 0.0;
+                    for (int c = 0; c < d; ++c) dsum += dog[c] * og[c];
+                    dd[(int64_t)h * T + t] = dsum;
+                }
+            }
+    }
     if (!rc) { P.row_sel = row_sel; rc = run_items(&P, 1, hq, nthreads); }   /* dQ rows */
     if (!rc) { P.row_sel = NULL; P.key_sel = key_sel; rc = run_items(&P, 2, hkv, nthreads); } /* dK, dV */
     if (!o_out) free(o);
     if (!lse_out) free(lse);
     free(dd);
     return rc;
+}
+
+/* The exact gradient of the forward definition (the oracle's own O and LSE). */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    const int32_t *cu_seqlens, int32_t nseq,
+                    int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                    const uint8_t *row_sel, const uint8_t *key_sel,
+                    double *dq, double *dk, double *dv,
+                    double *o_out, double *lse_out, int32_t nthreads)
+{
+    return oracle_attn_bwd_ex(q, k, v, dout, cu_seqlens, nseq, hq, hkv, d, scale, causal, row_sel, key_sel,
+                              NULL, NULL, dq, dk, dv, o_out, lse_out, nthreads);
 }
 
 /* The probability matrix of one (sequence, head) problem, materialised: p [n, n].

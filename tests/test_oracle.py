@@ -342,3 +342,42 @@ def test_thread_count_does_not_change_results():
     b = oracle.attn_bwd(q, k, v, do, cu, causal=True, threads=7)
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
+
+
+# ---------------------------------------------------------------------------------------
+# the backward as a function of its inputs (given O and LSE)
+# ---------------------------------------------------------------------------------------
+def test_backward_with_its_own_saved_outputs_is_unchanged():
+    lengths, hq, hkv, d = [13, 6], 4, 2, 5
+    T = sum(lengths)
+    cu = _cu(lengths)
+    q, k, v, do = _rand((T, hq, d), 60), _rand((T, hkv, d), 61), _rand((T, hkv, d), 62), _rand((T, hq, d), 63)
+    a = oracle.attn_bwd(q, k, v, do, cu, causal=True)
+    b = oracle.attn_bwd(q, k, v, do, cu, causal=True, o=a[3], lse=a[4])
+    for x, y in zip(a[:3], b[:3]):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-13)
+
+
+def test_given_lse_shift_scales_gradients_exactly():
+    """LSE + c gives P e^-c, so dV, dS and with them dQ, dK scale by e^-c (D comes from O)."""
+    T, hq, d = 17, 2, 4
+    q, k, v, do = _rand((T, hq, d), 64), _rand((T, hq, d), 65), _rand((T, hq, d), 66), _rand((T, hq, d), 67)
+    a = oracle.attn_bwd(q, k, v, do, causal=False)
+    c = 0.37
+    b = oracle.attn_bwd(q, k, v, do, causal=False, o=a[3], lse=a[4] + c)
+    for x, y in zip(a[:3], b[:3]):
+        np.testing.assert_allclose(y, x * math.exp(-c), rtol=1e-12, atol=1e-14)
+
+
+def test_given_o_changes_dq_by_closed_form():
+    """O + delta changes D_i by dO_i . delta_i; then dQ_i changes by
+    -scale * (dO_i . delta_i) * sum_j P_ij K_j, and sum_j P_ij K_j is the forward with V = K."""
+    T, hq, d = 15, 2, 3
+    scale = 0.8
+    q, k, v, do = _rand((T, hq, d), 68), _rand((T, hq, d), 69), _rand((T, hq, d), 70), _rand((T, hq, d), 71)
+    a = oracle.attn_bwd(q, k, v, do, scale=scale, causal=True)
+    delta = _rand((T, hq, d), 72, 1e-2)
+    b = oracle.attn_bwd(q, k, v, do, scale=scale, causal=True, o=a[3] + delta, lse=a[4])
+    pk, _ = oracle.attn_fwd(q, k, k, scale=scale, causal=True)
+    want = a[0] - scale * np.einsum("thc,thc->th", do, delta)[:, :, None] * pk
+    np.testing.assert_allclose(b[0], want, rtol=0, atol=1e-12)

@@ -27,6 +27,9 @@ MUTANTS = {
     "dV with Q in place of dO": ("av[c] += p[j] * doi[c];", "av[c] += p[j] * qi[c];"),
     "dQ with V in place of K": ("const double *kj = P->k + ((t0 + j) * P->hkv + g) * d;\n            for (int c = 0; c < d; ++c) dqi[c]",
                                 "const double *kj = P->v + ((t0 + j) * P->hkv + g) * d;\n            for (int c = 0; c < d; ++c) dqi[c]"),
+    "given LSE ignored": ("if (lse_in) lse[(int64_t)h * T + t] = lse_in[(int64_t)h * T + t];",
+                          "if (lse_in) lse[(int64_t)h * T + t] = lse[(int64_t)h * T + t];"),
+    "given O ignored for D": ("dd[(int64_t)h * T + t] = dsum;", "(void)dsum;"),
     "score mask boundary off by one": ("if (j >= vis) { s[j] = -INFINITY; continue; }", "if (j > vis) { s[j] = -INFINITY; continue; }"),
     "value row from the wrong key": ("const double *vj = P->v + ((key0 + j) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]",
                                      "const double *vj = P->v + ((key0 + (n - 1 - j)) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]"),
@@ -44,6 +47,8 @@ def _battery():
         lambda: pins.test_worked_example_online_merge(),
         lambda: pins.test_zero_queries_give_uniform_average(True),
         lambda: pins.test_gradient_invariants(False),
+        lambda: pins.test_given_lse_shift_scales_gradients_exactly(),
+        lambda: pins.test_given_o_changes_dq_by_closed_form(),
     ]
     for c in checks:
         try:
