@@ -38,16 +38,34 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 DATA = "synthetic: Q, K, V, dO iid N(0,1) drawn in fp32 from a seeded torch CPU generator, rounded to bf16"
 
 
+WORKLOAD = "mha2k"   # set from --workload
+
+
+def base_workload(name):
+    """The named workload (non-causal variant where it has both)."""
+    if name == "mha2k":
+        return W.mha2k(False)
+    if name.startswith("sweep_d"):       # sweep_d<d>_n<N>
+        d, n = name[len("sweep_d"):].split("_n")
+        return W.sweep(int(d), int(n))
+    return {"gqa8k": W.gqa8k(), "varlen16": W.varlen16(), "long32k": W.long32k()}[name]
+
+
 def workload_variants(rank=0):
-    base = W.mha2k(False)
-    base = W.Workload(base.name, base.batch, base.seqlen, base.hq, base.hkv, base.d, False, seed=base.seed + rank)
+    base = base_workload(WORKLOAD)
+    import dataclasses
+    base = dataclasses.replace(base, seed=base.seed + rank)
+    if base.causal:          # configurations that are causal only
+        return [base]
     return [base, base.with_causal(True)]
 
 
 def config_block(n_gpus):
-    w = W.mha2k(False)
-    return {"workload": f"mha2k: B={w.batch} H={w.hq} N={w.seqlen} d={w.d} bf16, fwd+bwd, non-causal and causal",
-            "global_batch": w.batch * n_gpus, "seq_len": w.seqlen, "heads": w.hq, "head_dim": w.d,
+    w = base_workload(WORKLOAD)
+    desc = (f"{WORKLOAD}: B={w.batch} Hq={w.hq} Hkv={w.hkv} N={w.seqlen or w.max_seqlen} d={w.d} bf16, fwd+bwd, "
+            + ("causal" if w.causal else "non-causal and causal"))
+    return {"workload": desc, "global_batch": w.batch * n_gpus, "seq_len": w.seqlen or w.max_seqlen,
+            "heads": w.hq, "head_dim": w.d,
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{n_gpus}"}
 
 
@@ -123,19 +141,21 @@ def oracle_sample(heads, budget_s=None):
     import oracle
     flops, secs, done = 0.0, 0.0, 0
     threads = oracle.default_threads()
-    base = workload_variants()[0]
+    variants = workload_variants()
+    base = variants[0]
     if "inputs" not in _ORACLE_CACHE:
         _ORACLE_CACHE["inputs"] = W.make_inputs(base)
-    q, k, v, do, _ = _ORACLE_CACHE["inputs"]
-    n = base.seqlen
+    q, k, v, do, cu = _ORACLE_CACHE["inputs"]
+    n = int(cu[1] - cu[0])
+    G = base.hq // base.hkv
     for h in range(base.hq):
         if heads is not None and done >= heads:
             break
         if budget_s is not None and secs >= budget_s:
             break
-        sl = (slice(0, n), slice(h, h + 1))
-        qs, ks, vs, dos = (t[sl].contiguous() for t in (q, k, v, do))
-        for causal in (False, True):
+        qs, dos = (t[:n, h:h + 1].contiguous() for t in (q, do))
+        ks, vs = (t[:n, h // G:h // G + 1].contiguous() for t in (k, v))
+        for causal in sorted({w.causal for w in variants}):
             t0 = time.perf_counter()
             oracle.attn_fwd(qs, ks, vs, scale=base.scale, causal=causal, threads=threads)
             oracle.attn_bwd(qs, ks, vs, dos, scale=base.scale, causal=causal, threads=threads)
@@ -158,7 +178,7 @@ def run_reference(args, rank, world):
         flops += f
         secs += s
     value = flops / secs / 1e12
-    sample = "fp64 CPU oracle, fwd+bwd of 1 head (N=2048, d=128) of sequence 0, non-causal and causal, per step"
+    sample = f"fp64 CPU oracle, fwd+bwd of 1 head of sequence 0 of {WORKLOAD} (all its mask variants), per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
@@ -193,24 +213,25 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     attn.load_library()
     variants = workload_variants(rank)
-    q, k, v, do, _ = W.make_inputs(variants[0])
+    q, k, v, do, cu = W.make_inputs(variants[0])
     host = {"q": q.pin_memory(), "k": k.pin_memory(), "v": v.pin_memory(), "do": do.pin_memory()}
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     w0 = variants[0]
+    shape_kw = (dict(cu_seqlens=cu.to(dev), max_seqlen=w0.max_seqlen) if w0.varlen else dict(batch=w0.batch))
     outs = {}
     for w in variants:
         outs[w.causal] = {"o": torch.empty_like(qd), "lse": torch.empty(w.hq, w.total_tokens, device=dev),
                           "dq": torch.empty_like(qd), "dk": torch.empty_like(kd), "dv": torch.empty_like(vd)}
-    ws = torch.empty(attn.workspace_size("bwd", qd, kd, batch=w0.batch), dtype=torch.uint8, device=dev)
+    ws = torch.empty(attn.workspace_size("bwd", qd, kd, **shape_kw), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
         for w in variants:
             b = outs[w.causal]
-            attn.attn_fwd(qd, kd, vd, scale=w.scale, causal=w.causal, batch=w.batch, o=b["o"], lse=b["lse"])
-            attn.attn_bwd(qd, kd, vd, b["o"], dod, b["lse"], scale=w.scale, causal=w.causal, batch=w.batch,
-                          dq=b["dq"], dk=b["dk"], dv=b["dv"], workspace=ws)
+            attn.attn_fwd(qd, kd, vd, scale=w.scale, causal=w.causal, o=b["o"], lse=b["lse"], **shape_kw)
+            attn.attn_bwd(qd, kd, vd, b["o"], dod, b["lse"], scale=w.scale, causal=w.causal,
+                          dq=b["dq"], dk=b["dk"], dv=b["dv"], workspace=ws, **shape_kw)
 
     def barrier():
         if world > 1:
@@ -257,9 +278,10 @@ def run_ours(args, rank, world, local_rank):
         return
     e2e_bufs = {}
     e2e_out = {}
+    host_kw = dict(cu_seqlens=cu, max_seqlen=w0.max_seqlen) if w0.varlen else dict(batch=w0.batch)
     for w in variants:
         _, e2e_bufs[w.causal] = attn.attention_host(host["q"], host["k"], host["v"], host["do"], scale=w.scale,
-                                                    causal=w.causal, batch=w.batch)
+                                                    causal=w.causal, **host_kw)
     torch.cuda.synchronize()
     h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "do")) * len(variants)
     d2h = sum(b["host_" + n].numel() * b["host_" + n].element_size()
@@ -270,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.steps):
         for w in variants:
             e2e_out[w.causal], _ = attn.attention_host(host["q"], host["k"], host["v"], host["do"], scale=w.scale,
-                                                       causal=w.causal, batch=w.batch, out=e2e_bufs[w.causal])
+                                                       causal=w.causal, out=e2e_bufs[w.causal], **host_kw)
     e2e_end.record(stream)
     barrier()
     attn.attn_get_device_error()
@@ -303,8 +325,8 @@ def run_ours(args, rank, world, local_rank):
     if world == 1:
         f, s, heads, threads = oracle_sample(heads=None, budget_s=12.0)
         cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"fp64 CPU oracle, fwd+bwd of {heads} whole head(s) (N=2048, d=128) of sequence 0, "
-                         f"non-causal and causal, {s:.1f} s"}
+               "sample": f"fp64 CPU oracle, fwd+bwd of {heads} whole head(s) of sequence 0 of {WORKLOAD} "
+                         f"(all its mask variants), {s:.1f} s"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config_block(world),
@@ -320,9 +342,13 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha2k",
+                    help="mha2k (the metric's configuration), sweep_d<d>_n<N>, gqa8k, varlen16 or long32k")
     ap.add_argument("--quick", action="store_true",
                     help="device timing only: skip the end-to-end loop and the CPU baseline (profiling runs)")
     args = ap.parse_args()
+    global WORKLOAD
+    WORKLOAD = args.workload
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -72,36 +72,48 @@ struct BwdCfg {
   static constexpr int Q_TILE_BYTES = BM * D * 2;
   static constexpr int DS_PANEL_BYTES = kKeys * 128;  // dS^T: 128 key rows x 64 queries (bf16)
   static constexpr int DS_BYTES = kKeys * BM * 2;
-  // TMEM columns
+  // TMEM columns.  d = 128: two dP^T buffers, so dP^T(n+1) can be issued before dK(n)
+  // reads dS^T(n) out of the other one, and a single dQ^T slot (its drain copies it out
+  // at once):  S^T [0,64) dP^T[0] [64,128) dP^T[1] [128,192) dV [192,320) dK [320,448)
+  // dQ^T [448,512).  d <= 64: one dP^T buffer and two dQ slots:
+  //   S^T [0,BM) dP^T [BM,2BM) dV, dK (d each) then two dQ slots of d columns.
+  static constexpr int NDPT = DQT ? 2 : 1;           // dP^T buffers
+  static constexpr int NDQ = DQT ? 1 : 2;            // dQ slots
   static constexpr int T_ST = 0;
-  static constexpr int T_DPT = BM;
-  static constexpr int T_DV = 2 * BM;
-  static constexpr int T_DK = 2 * BM + D;
-  static constexpr int T_DQ = 2 * BM + 2 * D;        // two buffers of DQ_COLS
+  static constexpr int T_DPT = BM;                   // dP^T buffer b at T_DPT + b * BM
+  static constexpr int T_DV = T_DPT + NDPT * BM;
+  static constexpr int T_DK = T_DV + D;
+  static constexpr int T_DQ = T_DK + D;              // NDQ slots of DQ_COLS
   static constexpr int DQ_COLS = DQT ? BM : D;
+  static_assert(T_DQ + NDQ * DQ_COLS <= 512, "TMEM budget");
   // shared memory map (offsets from the 1024-aligned base)
   static constexpr int O_K = 0;
   static constexpr int O_V = O_K + KV_TILE_BYTES;
   static constexpr int O_Q = O_V + KV_TILE_BYTES;              // STAGES
   static constexpr int O_DO = O_Q + STAGES * Q_TILE_BYTES;      // STAGES
   static constexpr int O_DS = O_DO + STAGES * Q_TILE_BYTES;     // 2 buffers
-  static constexpr int O_LSE = O_DS + 2 * DS_BYTES;            // STAGES x BM floats (LSE * log2 e)
-  static constexpr int O_DD = O_LSE + STAGES * BM * 4;         // STAGES x BM floats (D)
+  // LSE_i * log2 e and D_i rows live in LSLOTS slots (slot n % LSLOTS for step n), each
+  // with its own full barrier that the compute warpgroups observe phase by phase.
+  static constexpr int LSLOTS = 6;
+  static constexpr int O_LSE = O_DS + 2 * DS_BYTES;            // LSLOTS x BM floats
+  static constexpr int O_DD = O_LSE + LSLOTS * BM * 4;         // LSLOTS x BM floats
   // dQ staging tile for the bulk reduction, [BM query rows][d] fp32.  d = 128: plain
   // row-major (written column-wise, one feature per thread).  d <= 64: 32-float panels
   // with the 128-byte swizzle (written row-wise, one query row per thread).
   static constexpr int STG_ALIGN = DQT ? 128 : 1024;            // swizzled tiles need 1024
-  static constexpr int O_STG = (O_DD + STAGES * BM * 4 + STG_ALIGN - 1) & ~(STG_ALIGN - 1);
+  static constexpr int O_STG = (O_DD + LSLOTS * BM * 4 + STG_ALIGN - 1) & ~(STG_ALIGN - 1);
   static constexpr int STG_PANEL_BYTES = BM * 128;              // d <= 64: [BM rows][32 floats]
-  static constexpr int STG_BYTES = BM * D * 4;
+  static constexpr int STG_ROWS = DQT ? 32 : BM;                // d = 128: two halves of 32 rows
+  static constexpr int STG_BYTES = STG_ROWS * D * 4;
   static constexpr int O_BAR = O_STG + STG_BYTES;
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;                  // STAGES
   static constexpr int B_QEMPTY = B_QFULL + STAGES;  // STAGES
-  static constexpr int B_ST = B_QEMPTY + STAGES;
-  static constexpr int B_DPT = B_ST + 1;
-  static constexpr int B_PT = B_DPT + 1;
+  static constexpr int B_LFULL = B_QEMPTY + STAGES;  // LSLOTS
+  static constexpr int B_ST = B_LFULL + LSLOTS;
+  static constexpr int B_DPT = B_ST + 1;             // NDPT (2 slots reserved)
+  static constexpr int B_PT = B_DPT + 2;
   static constexpr int B_DS = B_PT + 1;
   static constexpr int B_DSFREE = B_DS + 1;          // 2
   static constexpr int B_DQFULL = B_DSFREE + 2;      // 2
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
-      if (i >= C::B_QFULL && i < C::B_QFULL + C::STAGES) cnt = 32;
+      if (i >= C::B_LFULL && i < C::B_LFULL + C::LSLOTS) cnt = 32;
       if (i == C::B_PT || i == C::B_DS) cnt = 256;
       if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 128;
       mbar_init(bar(i), cnt);
@@ -235,15 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     fetch(0);
     for (int n = 0; n < n_steps; ++n) {
       const int s = n % C::STAGES;
+      const int ls = n % C::LSLOTS;
+      // Stage s is free once dK(n - STAGES) is done; LSE slot ls was last read by step
+      // n - LSLOTS, whose dS finished before dK(n - LSLOTS), so it is free too.
       if (!mbar_wait(bar(C::B_QEMPTY + s), ((n / C::STAGES) & 1) ^ 1, abort_flag)) break;
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
 #pragma unroll
       for (int e = 0; e < PER_LANE; ++e) {
-        s_lse[s * BM + e * 32 + lane] = nl[e];
-        s_dd[s * BM + e * 32 + lane] = nd[e];
+        s_lse[ls * BM + e * 32 + lane] = nl[e];
+        s_dd[ls * BM + e * 32 + lane] = nd[e];
       }
+      mbar_arrive(bar(C::B_LFULL + ls));
       if (n + 1 < n_steps) fetch(n + 1);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
@@ -253,8 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sbase + C::O_DO + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmDO, bar(C::B_QFULL + s),
                       pn * C::PANEL, h, seq_start + q0);
         }
-      } else {
-        mbar_arrive(bar(C::B_QFULL + s));
       }
     }
   } else if (warp == 13) {
@@ -310,10 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_sdp(C::O_V, C::O_DO, C::T_DPT);
         mma_commit(bar(C::B_DPT));
       }
+      // Order per step n (dP^T buffer db = n & 1 when NDPT == 2, else 0):
+      //   [PT(n)] dV(n); S^T(n+1); NDPT == 2: dP^T(n+1) into the other buffer;
+      //   [DS(n)] dK(n) (reads dS^T(n) from buffer db); [dQ slot free] dQ(n);
+      //   NDPT == 1: dP^T(n+1) here, once dK(n) has been issued.
       for (int n = 0; ok && n < n_steps; ++n) {
         const int s = n % C::STAGES;
         const int s1 = (n + 1) % C::STAGES;
         const int b2 = n & 1;
+        const int db = C::NDPT == 2 ? b2 : 0;
+        const int db1 = C::NDPT == 2 ? (b2 ^ 1) : 0;
+        const int qslot = C::NDQ == 2 ? b2 : 0;
+        const uint32_t qpar = C::NDQ == 2 ? (((n >> 1) & 1) ^ 1) : (uint32_t)((n & 1) ^ 1);
         const uint32_t q_off = C::O_Q + s * C::Q_TILE_BYTES;
         const uint32_t do_off = C::O_DO + s * C::Q_TILE_BYTES;
         const bool more = n + 1 < n_steps;
@@ -325,17 +347,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           issue_sdp(C::O_K, C::O_Q + s1 * C::Q_TILE_BYTES, C::T_ST);   // S^T for the next step
           mma_commit(bar(C::B_ST));
+          if (C::NDPT == 2) {
+            issue_sdp(C::O_V, C::O_DO + s1 * C::Q_TILE_BYTES, C::T_DPT + db1 * BM);   // dP^T(n+1)
+            mma_commit(bar(C::B_DPT + db1));
+          }
         }
         if (!mbar_wait(bar(C::B_DS), n & 1, abort_flag)) break;
         tc_fence_after();
-        issue_grad(C::T_DPT, q_off, C::T_DK, n > 0);                  // dK += dS^T Q
+        issue_grad(C::T_DPT + db * BM, q_off, C::T_DK, n > 0);        // dK += dS^T Q
         mma_commit(bar(C::B_QEMPTY + s));
-        if (!mbar_wait(bar(C::B_DQEMPTY + b2), ((n >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) break;
         tc_fence_after();
-        issue_dq(b2, C::T_DQ + b2 * C::DQ_COLS);                       // dQ_i partial
-        mma_commit(bar(C::B_DQFULL + b2));
+        issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                    // dQ_i partial
+        mma_commit(bar(C::B_DQFULL + qslot));
         mma_commit(bar(C::B_DSFREE + b2));
-        if (more) {
+        if (C::NDPT == 1 && more) {
           issue_sdp(C::O_V, C::O_DO + s1 * C::Q_TILE_BYTES, C::T_DPT);  // dP^T for the next step
           mma_commit(bar(C::B_DPT));
         }
@@ -353,8 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int n = 0; n < n_steps; ++n) {
-      const int s = n % C::STAGES;
+      const int ls = n % C::LSLOTS;
       const int b2 = n & 1;
+      const int db = C::NDPT == 2 ? b2 : 0;                           // dP^T buffer
+      const uint32_t dpar = C::NDPT == 2 ? ((n >> 1) & 1) : (uint32_t)(n & 1);
+      const uint32_t t_dpt = C::T_DPT + db * BM;
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
@@ -363,11 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int c_lo = p.causal ? kj - q0 : 0;
       if (kj >= len) c_lo = BM;
       const bool masked = c_lo > c0;
-      if (!mbar_wait(bar(C::B_QFULL + s), (n / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_LFULL + ls), (n / C::LSLOTS) & 1, abort_flag)) { ok = false; break; }
       if (!mbar_wait(bar(C::B_ST), n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const float4* lse4 = reinterpret_cast<const float4*>(s_lse + s * BM + c0);
-      const float4* dd4 = reinterpret_cast<const float4*>(s_dd + s * BM + c0);
+      const float4* lse4 = reinterpret_cast<const float4*>(s_lse + ls * BM + c0);
+      const float4* dd4 = reinterpret_cast<const float4*>(s_dd + ls * BM + c0);
       float pr[HALF];
 #pragma unroll
       for (int cb = 0; cb < HALF; cb += 32) {
@@ -402,13 +431,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(C::B_PT));
       // dS^T = P^T o (dP^T - D): to TMEM (over dP^T) and to the swizzled SMEM buffer
       if (!mbar_wait(bar(C::B_DSFREE + b2), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(C::B_DPT), n & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_DPT + db), dpar, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint8_t* ds_smem = smem + C::O_DS + b2 * C::DS_BYTES;
 #pragma unroll
       for (int cb = 0; cb < HALF; cb += 32) {
         uint32_t r[32];
-        tmem_ld32(trow + C::T_DPT + c0 + cb, r);
+        tmem_ld32(trow + t_dpt + c0 + cb, r);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
@@ -420,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           w[2 * e4 + 1] = pack_bf16x2(pr[cb + e + 2] * (__uint_as_float(r[e + 2]) - d4.z),
                                       pr[cb + e + 3] * (__uint_as_float(r[e + 3]) - d4.w));
         }
-        tmem_st16(trow + C::T_DPT + c0 + cb / 2, w);
+        tmem_st16(trow + t_dpt + c0 + cb / 2, w);
         // queries c0+cb .. +31 live in panel (c0+cb)/64, 16-byte chunks ((c0+cb)%64)/8 .. +3
         uint8_t* panel = ds_smem + ((c0 + cb) / 64) * C::DS_PANEL_BYTES;
 #pragma unroll
@@ -464,11 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane_base = (warp & 3) * 32;
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     for (int n = 0; n < n_steps; ++n) {
-      const int b2 = n & 1;
+      const int b2 = C::NDQ == 2 ? (n & 1) : 0;                    // dQ slot
+      const uint32_t par = C::NDQ == 2 ? ((n >> 1) & 1) : (uint32_t)(n & 1);
       int h, i;
       it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
-      if (!mbar_wait(bar(C::B_DQFULL + b2), (n >> 1) & 1, abort_flag)) break;
+      if (!mbar_wait(bar(C::B_DQFULL + b2), par, abort_flag)) break;
       tc_fence_after();
       uint32_t r[C::DQ_COLS / 32][32];
 #pragma unroll
@@ -481,16 +511,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // transposed into a [BM][d] fp32 staging tile and added into the accumulator by
         // one bulk tensor reduction (query rows past the sequence carry exact zeros).
         const int c = lane_base + lane;
-        if (warp == 8 && lane == 0) bulk_wait_group_read0();   // previous reduce has read the tile
-        named_barrier_sync(1, 128);
         float* stg = reinterpret_cast<float*>(smem + C::O_STG);
 #pragma unroll
-        for (int e = 0; e < BM; ++e) stg[e * D + c] = __uint_as_float(r[e / 32][e % 32]);
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (warp == 8 && lane == 0) {
-          tma_reduce_add_3d(&tmDQ, sbase + C::O_STG, 0, h, seq_start + q0);
-          bulk_commit_group();
+        for (int part = 0; part < BM / C::STG_ROWS; ++part) {
+          if (warp == 8 && lane == 0) bulk_wait_group_read0();   // previous reduce has read the tile
+          named_barrier_sync(1, 128);
+#pragma unroll
+          for (int e = 0; e < C::STG_ROWS; ++e) {
+            const int row = part * C::STG_ROWS + e;
+            stg[e * D + c] = __uint_as_float(r[row / 32][row % 32]);
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1, 128);
+          if (warp == 8 && lane == 0) {
+            tma_reduce_add_3d(&tmDQ, sbase + C::O_STG, 0, h, seq_start + q0 + part * C::STG_ROWS);
+            bulk_commit_group();
+          }
         }
       } else {
         // lane = query row, registers = its d features.  Each 32-feature panel row is 128
@@ -618,7 +654,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
     if (e != cudaSuccess) return e;
   }
   alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!encode_tma_3d_f32(&tdq, dq_acc, D, pb.hq, pb.total_tokens, C::DQT ? D : 32, C::BM) ||
+  if (!encode_tma_3d_f32(&tdq, dq_acc, D, pb.hq, pb.total_tokens, C::DQT ? D : 32, C::STG_ROWS) ||
       !encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
       !encode_tma_3d(&tdo, dout, D, pb.hq, pb.total_tokens, C::PANEL, C::BM) ||
       !encode_tma_3d(&tk, k, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys) ||
