@@ -194,9 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
-      if (i >= C::B_LFULL && i < C::B_LFULL + C::LSLOTS) cnt = 32;
-      if (i == C::B_PT || i == C::B_DS) cnt = 256;
-      if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 128;
+      // warp-level arrivals: one per compute warp (PT, DS) or drain warp (DQEMPTY)
+      if (i == C::B_PT || i == C::B_DS) cnt = 8;
+      if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 4;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_lse[ls * BM + e * 32 + lane] = nl[e];
         s_dd[ls * BM + e * 32 + lane] = nd[e];
       }
-      mbar_arrive(bar(C::B_LFULL + ls));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_LFULL + ls));
       if (n + 1 < n_steps) fetch(n + 1);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
@@ -428,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PT));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PT));
       // dS^T = P^T o (dP^T - D): to TMEM (over dP^T) and to the swizzled SMEM buffer
       if (!mbar_wait(bar(C::B_DSFREE + b2), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       if (!mbar_wait(bar(C::B_DPT + db), dpar, abort_flag)) { ok = false; break; }
@@ -462,7 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DS));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_DS));
     }
     // ---------------- epilogue: warps 0-3 write dV, warps 4-7 write dK = scale * acc ------
     if (ok && mbar_wait(bar(C::B_DONE), 0, abort_flag)) {
@@ -505,7 +508,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cb = 0; cb < C::DQ_COLS / 32; ++cb) tmem_ld32(trow + C::T_DQ + b2 * C::DQ_COLS + cb * 32, r[cb]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DQEMPTY + b2));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_DQEMPTY + b2));
       if (C::DQT) {
         // lane = feature c, registers = the BM query rows of this step.  The partial is
         // transposed into a [BM][d] fp32 staging tile and added into the accumulator by

@@ -5,9 +5,9 @@
 // tutorial, sections 标准注意力三步 and 前向).
 //
 // How (sections 分块, Online Softmax 技巧 and 伪代码骨架 of the same tutorial; FA2's
-// query-outer loop order from the "Flash-Attention" concept page, 核心思想): each CTA owns
-// two 128-row query tiles of one head and streams the sequence's 128-key K/V tiles
-// through shared memory once.  Per key tile and query tile t:
+// query-outer loop order from the "Flash-Attention" concept page, 核心思想): a work item
+// is two 128-row query tiles of one head; the item streams the sequence's 128-key K/V
+// tiles through shared memory once.  Per key tile and query tile t:
 //     S_t   = Q_t K_j^T                  tcgen05 MMA, A and B from swizzled SMEM, fp32 in TMEM
 //     m_new = max(m_old, rowmax(S_t))    one query row per thread, no shuffles
 //     P_t   = exp2(S_t * scale*log2e - m_new), l = l * exp2(m_old - m_new) + rowsum(P_t)
@@ -23,13 +23,22 @@
 // consistently, so the result is exact up to rounding.  (The concept page lists this
 // "conditional rescaling" among the Blackwell techniques, 已知局限.)
 //
+// Persistent schedule: one CTA per SM walks a static list of work items, heaviest first
+// under the causal mask (zig-zag over CTAs so every CTA gets a similar total), pairs of one
+// head adjacent otherwise (their K/V stream is shared through L2).  All pipelines run
+// across items: the next item's Q load and its first QK^T MMAs overlap the current item's
+// epilogue, and the K/V ring never drains.  Under the causal mask a query tile only
+// visits key tiles it can see, so the lower tile of an item skips the last key tile.
+//
 // Warp roles (320 threads):
 //   warps 0-3  softmax + correction + epilogue for query tile 0 (TMEM lanes 0..127)
 //   warps 4-7  the same for query tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j / V_j into a STAGES-deep ring
+//   warp  8    TMA producer: Q tiles per item, K_j / V_j into a STAGES-deep ring
 //   warp  9    MMA issuer (one thread): S0, S1, then PV0, S0', PV1, S1', ... so the tensor
 //              core works on one tile while the other tile's softmax runs.
 // TMEM (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 after.
+#include <algorithm>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -40,6 +49,10 @@ namespace {
 constexpr int kRows = 128;                 // query rows per tile == TMEM lanes
 constexpr int kKeys = 128;                 // keys per K/V tile
 constexpr float kRescaleSkip = 8.0f;       // log2 units, see file comment
+// Pairs of exponentials computed on the FMA pipe in unmasked tiles: bit (c % 8) of this
+// mask selects pair c (2 of every 8 pairs, 25%, the best of 0 / 25 / 37.5 / 50% measured
+// on B200), balancing the special-function unit against the FMA pipe.
+constexpr uint32_t kEmuPairs = 0x22u;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
 
@@ -55,28 +68,77 @@ struct FwdCfg {
   static constexpr int SBO = 8 * SW;               // bytes between 8-row swizzle atoms
   static constexpr int KSTEPS_PER_PANEL = SW / 32; // 16-element K steps inside one panel
   // barrier slots
-  static constexpr int B_Q = 0;
-  static constexpr int B_KFULL = 1;
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_QEMPTY = 1;
+  static constexpr int B_KFULL = 2;
   static constexpr int B_VFULL = B_KFULL + STAGES;
   static constexpr int B_KEMPTY = B_VFULL + STAGES;
   static constexpr int B_VEMPTY = B_KEMPTY + STAGES;
   static constexpr int B_SFULL = B_VEMPTY + STAGES;  // 2
   static constexpr int B_PFULL = B_SFULL + 2;        // 2
   static constexpr int B_OFINAL = B_PFULL + 2;       // 2
-  static constexpr int NBARS = B_OFINAL + 2;
+  static constexpr int B_OFREE = B_OFINAL + 2;       // 2
+  static constexpr int NBARS = B_OFREE + 2;
   static constexpr int DATA_BYTES = (2 + 2 * STAGES) * TILE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 16;
 };
 
 struct FwdParams {
   const int32_t* cu_seqlens;
-  int32_t seqlen, max_seqlen, total_tokens, hq, hkv;
+  int32_t seqlen, max_seqlen, total_tokens, hq, hkv, batch;
+  int32_t n_pairs, n_items;
   float scale_log2;  // scale * log2(e), rounded to fp32
   double lse_skew;   // scale_log2 * ln 2 - scale, in double: the rounding of scale_log2
   int32_t causal;
   __nv_bfloat16* o;
   float* lse;
 };
+
+// One work item: two query tiles of one head of one sequence.
+struct Item {
+  int h, b, seq_start, len, q0;
+  int n[2];    // key tiles each query tile visits (0: the tile is past the sequence)
+  int nkv;     // key tiles loaded for the item, max(n[0], n[1])
+};
+
+__device__ __forceinline__ Item make_item(const FwdParams& p, int k) {
+  // k-th item of this CTA.  Causal: heaviest first, zig-zag over CTAs.  Otherwise the
+  // pairs of one head are consecutive.
+  const int G = gridDim.x;
+  const int idx = k * G + ((p.causal && (k & 1)) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+  Item it;
+  if (idx >= p.n_items) {   // the last round is partial
+    it.h = it.b = it.seq_start = it.len = it.q0 = 0;
+    it.n[0] = it.n[1] = it.nkv = 0;
+    return it;
+  }
+  int pair;
+  if (p.causal) {
+    it.h = idx % p.hq;
+    const int t = idx / p.hq;
+    it.b = t % p.batch;
+    pair = p.n_pairs - 1 - t / p.batch;
+  } else {
+    pair = idx % p.n_pairs;
+    const int t = idx / p.n_pairs;
+    it.h = t % p.hq;
+    it.b = t / p.hq;
+  }
+  it.seq_start = p.cu_seqlens ? p.cu_seqlens[it.b] : it.b * p.seqlen;
+  it.len = p.cu_seqlens ? p.cu_seqlens[it.b + 1] - it.seq_start : p.seqlen;
+  it.q0 = pair * 2 * kRows;
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = it.q0 + t * kRows;
+    if (r0 >= it.len) {
+      it.n[t] = 0;
+    } else {
+      const int kv_end = p.causal ? min(it.len, r0 + kRows) : it.len;
+      it.n[t] = (kv_end + kKeys - 1) / kKeys;
+    }
+  }
+  it.nkv = max(it.n[0], it.n[1]);
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -96,34 +158,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Launch order.  Without a mask every CTA does the same work, and the query-tile pairs
-  // of one head are adjacent (grid x) so their shared K/V stream is served from L2.  With
-  // the causal mask the work grows with the pair index, so the heaviest pairs of every
-  // head go first (grid z, reversed) to keep the tail of the launch short.
-  int pair, h, b;
-  if (p.causal) {
-    h = blockIdx.x;
-    b = blockIdx.y;
-    pair = gridDim.z - 1 - blockIdx.z;
-  } else {
-    pair = blockIdx.x;
-    h = blockIdx.y;
-    b = blockIdx.z;
-  }
-  const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
-  const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
-  if (len > p.max_seqlen) {
-    if (threadIdx.x == 0 && pair == 0 && h == 0) report_error(ATTN_DEVERR_SEQLEN);
-  }
-  const int q0 = pair * 2 * kRows;
-  if (q0 >= len) return;   // uniform over the CTA, before any barrier or TMEM use
-  const int kv_end = p.causal ? min(len, q0 + 2 * kRows) : len;
-  const int n_kv = (kv_end + kKeys - 1) / kKeys;
+  // Every CTA walks the same number of rounds; indices past the item list are empty items.
+  const int n_mine = (p.n_items + (int)gridDim.x - 1) / (int)gridDim.x;
 
   if (threadIdx.x == 0) {
+    // sequences longer than max_seqlen would not be covered by the item list
+    if (blockIdx.x == 0)
+      for (int b = 0; b < p.batch; ++b) {
+        const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - p.cu_seqlens[b] : p.seqlen;
+        if (len > p.max_seqlen) report_error(ATTN_DEVERR_SEQLEN);
+      }
     for (int i = 0; i < C::NBARS; ++i) {
-      const bool per_thread = (i == C::B_PFULL || i == C::B_PFULL + 1);
-      mbar_init(bar(i), per_thread ? 128u : 1u);
+      // P-ready and O-free are arrived on once per softmax warp (after __syncwarp)
+      const bool per_warp = (i == C::B_PFULL || i == C::B_PFULL + 1 || i == C::B_OFREE || i == C::B_OFREE + 1);
+      mbar_init(bar(i), per_warp ? 4u : 1u);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -145,25 +193,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      const int hk = h / (p.hq / p.hkv);
-      mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::TILE_BYTES);
-      for (int t = 0; t < 2; ++t)
-        for (int pn = 0; pn < C::NPANEL; ++pn)
-          tma_load_3d(sQ + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, bar(C::B_Q), pn * C::PANEL, h,
-                      seq_start + q0 + t * kRows);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        if (!mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
-        for (int pn = 0; pn < C::NPANEL; ++pn)
-          tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, hk,
-                      seq_start + j * kKeys);
-        if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
-        for (int pn = 0; pn < C::NPANEL; ++pn)
-          tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, hk,
-                      seq_start + j * kKeys);
+      uint32_t kv = 0, qi = 0;   // K/V tiles and non-empty items so far
+      bool ok = true;
+      for (int k = 0; ok && k < n_mine; ++k) {
+        const Item it = make_item(p, k);
+        if (it.nkv == 0) continue;
+        const int hk = it.h / (p.hq / p.hkv);
+        if (!mbar_wait(bar(C::B_QEMPTY), (qi & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_QFULL), ((it.n[0] > 0) + (it.n[1] > 0)) * C::TILE_BYTES);
+        for (int t = 0; t < 2; ++t)
+          if (it.n[t] > 0)
+            for (int pn = 0; pn < C::NPANEL; ++pn)
+              tma_load_3d(sQ + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, bar(C::B_QFULL), pn * C::PANEL, it.h,
+                          it.seq_start + it.q0 + t * kRows);
+        for (int j = 0; j < it.nkv; ++j, ++kv) {
+          const int s = kv % C::STAGES;
+          const uint32_t ph = (kv / C::STAGES) & 1;
+          if (!mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, hk,
+                        it.seq_start + j * kKeys);
+          if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, hk,
+                        it.seq_start + j * kKeys);
+        }
+        ++qi;
       }
     }
   } else if (warp == 9) {
@@ -190,143 +247,204 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(d_tmem, a_tmem, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag) && mbar_wait(bar(C::B_KFULL), 0, abort_flag);
-      if (ok) {
+      uint32_t kv = 0, qi = 0;
+      uint32_t pc[2] = {0, 0};   // P_t tiles consumed
+      uint32_t om[2] = {0, 0};   // items started per query tile (for the O-free handshake)
+      bool ok = true;
+      for (int k = 0; ok && k < n_mine; ++k) {
+        const Item it = make_item(p, k);
+        if (it.nkv == 0) continue;
+        int s_left = it.n[0] + it.n[1];   // QK^T MMAs still to issue; Q is free after the last
+        ok = mbar_wait(bar(C::B_QFULL), qi & 1, abort_flag);
+        const int s0 = kv % C::STAGES;
+        ok = ok && mbar_wait(bar(C::B_KFULL + s0), (kv / C::STAGES) & 1, abort_flag);
+        if (!ok) break;
         tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(bar(C::B_SFULL + 0));
-        issue_qk(1, 0);
-        mma_commit(bar(C::B_SFULL + 1));
-        mma_commit(bar(C::B_KEMPTY + 0));
-      }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        const bool more = j + 1 < n_kv;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-        if (!mbar_wait(bar(C::B_VFULL + s), ph, abort_flag)) break;
-        if (!mbar_wait(bar(C::B_PFULL + 0), j & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_pv(0, s, j > 0);
-        if (more) {
-          if (!mbar_wait(bar(C::B_KFULL + s1), ph1, abort_flag)) break;
-          tc_fence_after();
-          issue_qk(0, s1);
-          mma_commit(bar(C::B_SFULL + 0));
-        } else {
-          mma_commit(bar(C::B_OFINAL + 0));
+        for (int t = 0; t < 2; ++t)
+          if (it.n[t] > 0) {
+            issue_qk(t, s0);
+            mma_commit(bar(C::B_SFULL + t));
+            if (--s_left == 0) mma_commit(bar(C::B_QEMPTY));
+          }
+        mma_commit(bar(C::B_KEMPTY + s0));
+        for (int j = 0; ok && j < it.nkv; ++j) {
+          const uint32_t c = kv + j;
+          const int s = c % C::STAGES;
+          if (!mbar_wait(bar(C::B_VFULL + s), (c / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+          bool k_next = false;
+          const int s1 = (c + 1) % C::STAGES;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= it.n[t]) continue;
+            if (!mbar_wait(bar(C::B_PFULL + t), pc[t] & 1, abort_flag)) { ok = false; break; }
+            ++pc[t];
+            if (j == 0) {   // O_t of the previous item has been read out
+              if (!mbar_wait(bar(C::B_OFREE + t), (om[t] & 1) ^ 1, abort_flag)) { ok = false; break; }
+              ++om[t];
+            }
+            tc_fence_after();
+            issue_pv(t, s, j > 0);
+            if (j + 1 < it.n[t]) {
+              if (!k_next) {
+                if (!mbar_wait(bar(C::B_KFULL + s1), ((c + 1) / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                k_next = true;
+              }
+              issue_qk(t, s1);
+              mma_commit(bar(C::B_SFULL + t));
+              if (--s_left == 0) mma_commit(bar(C::B_QEMPTY));
+            } else {
+              mma_commit(bar(C::B_OFINAL + t));
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar(C::B_VEMPTY + s));
+          if (k_next) mma_commit(bar(C::B_KEMPTY + s1));
         }
-        if (!mbar_wait(bar(C::B_PFULL + 1), j & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_pv(1, s, j > 0);
-        mma_commit(bar(C::B_VEMPTY + s));
-        if (more) {
-          issue_qk(1, s1);
-          mma_commit(bar(C::B_SFULL + 1));
-          mma_commit(bar(C::B_KEMPTY + s1));
-        } else {
-          mma_commit(bar(C::B_OFINAL + 1));
-        }
+        kv += it.nkv;
+        ++qi;
       }
     }
   } else {
     // ---------------- softmax / correction / epilogue (one query row per thread) ---------
     const int t = warp >> 2;                        // query tile of this warpgroup
     const int lane_base = (warp & 3) * 32;          // TMEM lanes this warp may touch
-    const int qi = q0 + t * kRows + lane_base + lane;   // query index inside the sequence
     const uint32_t tS = tmem + ((uint32_t)lane_base << 16) + t * kKeys;
     const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + 2 * kKeys + t * D;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY;   // running max in log2 units (possibly stale by < 8)
-    float mx_used = 0.f;        // the raw score maximum that m_used was formed from
-    float l = 0.f;              // running sum of exp2(x - m_used)
+    uint32_t sc = 0, oc = 0;   // S_t tiles and items consumed by this warpgroup
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(bar(C::B_SFULL + t), j & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      float s[kKeys];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS + 0, r0);
-        tmem_ld32(tS + 32, r1);
-        tmem_ld32(tS + 64, r2);
-        tmem_ld32(tS + 96, r3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = __uint_as_float(r0[c]);
-          s[32 + c] = __uint_as_float(r1[c]);
-          s[64 + c] = __uint_as_float(r2[c]);
-          s[96 + c] = __uint_as_float(r3[c]);
-        }
-      }
-      // mask: key kbase + c is visible iff it is inside the sequence and, when causal,
-      // not after this query.
-      const int kbase = j * kKeys;
-      int lim = len - 1 - kbase;
-      if (p.causal) lim = min(lim, qi - kbase);
-      if (lim < kKeys - 1) {
-#pragma unroll
-        for (int c = 0; c < kKeys; ++c)
-          if (c > lim) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
-      float m_new = m_used;
-      if (m_cand > m_used + kRescaleSkip) {
-        m_new = m_cand;
-        mx_used = mx;
-      }
-      const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
-      float rowsum = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(fmaf(s[2 * c], sl2, -m_sub));
-        const float p1 = ex2(fmaf(s[2 * c + 1], sl2, -m_sub));
-        rowsum += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(tS + 0, lo);
-        tmem_st32(tS + 32, hi);
-      }
-      float alpha = 1.f;
-      if (m_new != m_used) {
-        alpha = ex2(m_used - m_sub);   // 0 when m_used is -inf
-        l = l * alpha + rowsum;
-      } else {
-        l += rowsum;
-      }
-      const bool need = (j > 0) && (m_new != m_used);
-      m_used = m_new;
-      if (__any_sync(0xffffffffu, need)) {
-        // O_t was last written by PV_t(j-1), which completed before S_t(j) was signalled.
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
+    for (int k = 0; ok && k < n_mine; ++k) {
+      const Item it = make_item(p, k);
+      const int n_t = it.n[t];
+      if (n_t == 0) continue;
+      const int qi = it.q0 + t * kRows + lane_base + lane;   // query index inside the sequence
+      float m_used = -INFINITY;   // running max in log2 units (possibly stale by < 8)
+      float mx_used = 0.f;        // the raw score maximum that m_used was formed from
+      float l = 0.f;              // running sum of exp2(x - m_used)
+      for (int j = 0; j < n_t; ++j) {
+        if (!mbar_wait(bar(C::B_SFULL + t), sc & 1, abort_flag)) { ok = false; break; }
+        ++sc;
+        tc_fence_after();
+        float s[kKeys];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS + 0, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tO + c * 32, r);
+          for (int c = 0; c < 32; ++c) {
+            s[c] = __uint_as_float(r0[c]);
+            s[32 + c] = __uint_as_float(r1[c]);
+            s[64 + c] = __uint_as_float(r2[c]);
+            s[96 + c] = __uint_as_float(r3[c]);
+          }
         }
+        // mask: key kbase + c is visible iff it is inside the sequence and, when causal,
+        // not after this query.
+        const int kbase = j * kKeys;
+        int lim = it.len - 1 - kbase;
+        if (p.causal) lim = min(lim, qi - kbase);
+        const bool masked = lim < kKeys - 1;
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c)
+            if (c > lim) s[c] = -INFINITY;
+        }
+        // Row max over 8 independent partial maxima (short dependency chains).
+        float mp[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mp[a] = fmaxf(s[a], s[8 + a]);
+#pragma unroll
+        for (int c = 16; c < kKeys; c += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mp[a] = max3(mp[a], s[c + a], s[c + 8 + a]);
+        const float mx = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        const float m_cand = mx * sl2;
+        float m_new = m_used;
+        if (m_cand > m_used + kRescaleSkip) {
+          m_new = m_cand;
+          mx_used = mx;
+        }
+        const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
+        uint32_t pk[64];
+        const uint64_t sl2x2 = f2(sl2, sl2);
+        const uint64_t negm = f2(-m_sub, -m_sub);
+        uint64_t sum2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // 8 partial sums
+        if (masked) {
+          // hidden keys must come out as exact zeros: special-function unit only
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float x0, x1;
+            f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sl2x2, negm), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            sum2[c & 3] = add2(sum2[c & 3], f2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // A share of the exponentials (the pairs c with bit c % 8 set in kEmuPairs) runs
+          // on the FMA pipe, the rest on the special-function unit, so the two units share
+          // the row's exponential work.
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const uint64_t x = fma2(f2(s[2 * c], s[2 * c + 1]), sl2x2, negm);
+            float p0, p1;
+            if ((kEmuPairs >> (c % 8)) & 1u) {
+              ex2_fma_pair(x, p0, p1);
+            } else {
+              float x0, x1;
+              f2_split(x, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            sum2[c & 3] = add2(sum2[c & 3], f2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+        }
+        float sum_lo, sum_hi;
+        f2_split(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])), sum_lo, sum_hi);
+        const float rowsum = sum_lo + sum_hi;
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+          tmem_st32(tS + 0, lo);
+          tmem_st32(tS + 32, hi);
+        }
+        float alpha = 1.f;
+        if (m_new != m_used) {
+          alpha = ex2(m_used - m_sub);   // 0 when m_used is -inf
+          l = l * alpha + rowsum;
+        } else {
+          l += rowsum;
+        }
+        const bool need = (j > 0) && (m_new != m_used);
+        m_used = m_new;
+        if (__any_sync(0xffffffffu, need)) {
+          // O_t was last written by PV_t(j-1), which completed before S_t(j) was signalled.
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tO + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_PFULL + t));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + t));
-    }
-    // ---------------- epilogue: O / l and LSE ----------------
-    if (ok && mbar_wait(bar(C::B_OFINAL + t), 0, abort_flag)) {
+      if (!ok) break;
+      // ---------------- epilogue: O / l and LSE, then hand O_t back to the MMA ----------------
+      if (!mbar_wait(bar(C::B_OFINAL + t), oc & 1, abort_flag)) { ok = false; break; }
+      ++oc;
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const bool row_ok = qi < len;
-      __nv_bfloat16* orow = p.o + ((size_t)(seq_start + qi) * p.hq + h) * D;
+      const bool row_ok = qi < it.len;
+      __nv_bfloat16* orow = p.o + ((size_t)(it.seq_start + qi) * p.hq + it.h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -342,6 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_OFREE + t));
       if (row_ok) {
         // LSE = m ln 2 + ln l, evaluated in double from the exact fp32 values the
         // exponentials used (m_used, l), minus the first-order effect of scale_log2 being
@@ -349,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lse = -INFINITY;
         if (l > 0.f)
           lse = (float)((double)m_used * 0.6931471805599453 + log((double)l) - p.lse_skew * (double)mx_used);
-        p.lse[(size_t)h * p.total_tokens + seq_start + qi] = lse;
+        p.lse[(size_t)it.h * p.total_tokens + it.seq_start + qi] = lse;
       }
     }
   }
@@ -360,6 +481,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+int sm_count_fwd() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
 }
 
 template <int D>
@@ -378,6 +509,11 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   p.total_tokens = pb.total_tokens;
   p.hq = pb.hq;
   p.hkv = pb.hkv;
+  p.batch = pb.batch;
+  p.n_pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
+  const int64_t items = (int64_t)p.n_pairs * pb.hq * pb.batch;
+  if (items > INT32_MAX) return cudaErrorInvalidValue;
+  p.n_items = (int)items;
   p.scale_log2 = pb.scale * kLog2e;
   p.lse_skew = (double)p.scale_log2 * 0.6931471805599453 - (double)pb.scale;
   p.causal = pb.causal;
@@ -385,8 +521,7 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   p.lse = lse;
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
-  const dim3 grid = pb.causal ? dim3(pb.hq, pb.batch, pairs) : dim3(pairs, pb.hq, pb.batch);
+  const int grid = (int)std::min<int64_t>(items, sm_count_fwd());
   LaunchScope scope(K_FWD_BF16, stream);
   fwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

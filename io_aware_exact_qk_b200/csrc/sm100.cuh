@@ -237,6 +237,60 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// ---- packed fp32 pairs (sm_100 f32x2 instructions: one issue slot for two lanes' worth) ----
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of x, computed on the FMA pipe instead of the special-function unit, so
+// that part of a softmax row's exponentials can run beside the others.  Method (a
+// Cody-Waite style range reduction): x is clamped to >= -125, split as x = n + f with
+// n = round(x) obtained by adding 1.5 * 2^23 (which leaves n in the low mantissa bits),
+// f = x - n in [-0.5, 0.5]; 2^f comes from a cubic whose coefficients were fitted to 2^f
+// on [-0.5, 0.5] by least squares on the relative error, reweighted toward the largest
+// errors (max relative error 7.5e-5 in fp32 Horner form); 2^n is applied by adding n to
+// the exponent field.  Valid for x <= 127 (the softmax passes x <= 8).
+__device__ __forceinline__ void ex2_fma_pair(uint64_t x, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;          // 1.5 * 2^23
+  float x0, x1;
+  f2_split(x, x0, x1);
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const uint64_t xc = f2(x0, x1);
+  const uint64_t t = add2(xc, f2(kShift, kShift));            // n + 1.5 * 2^23
+  const uint64_t r = add2(t, f2(-kShift, -kShift));           // n as a float
+  const uint64_t fr = fma2(r, f2(-1.0f, -1.0f), xc);          // f = x - n
+  uint64_t q = fma2(f2(0.05517097935f, 0.05517097935f), fr, f2(0.24260970950f, 0.24260970950f));
+  q = fma2(q, fr, f2(0.69326096773f, 0.69326096773f));
+  q = fma2(q, fr, f2(0.99992817640f, 0.99992817640f));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  // t's bit pattern is 0x4B400000 + n, so (bits(t) << 23) == n << 23 modulo 2^32
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // Two floats -> packed bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
