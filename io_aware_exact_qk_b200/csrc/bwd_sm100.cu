@@ -32,8 +32,8 @@
 // the CTA that owns the key tile adds it into an fp32 accumulator with atomics.  The
 // alternative -- a second, query-major kernel -- would recompute S and dP (7 matrix
 // products per tile instead of 5, 40% more tensor work); the atomic traffic instead goes
-// to L2 (the accumulator of one head, N*d*4 bytes, stays L2-resident), coalesced
-// 128 bytes per warp instruction (d = 128) or 16-byte vector atomics (d <= 64).
+// to L2 (the accumulator of one head, N*d*4 bytes, stays L2-resident): the drain stages
+// each partial in an fp32 SMEM tile and adds it with bulk tensor reductions.
 //
 // TMEM shapes.  d = 128 uses BM = 64 query rows per step and forms the transpose
 // dQ_i^T = K_j^T dS^T (M = d = 128, N = 64), which fits S^T (64) + dP^T (64) + dV (128)
@@ -57,7 +57,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D>
 struct BwdCfg {
   static constexpr bool DQT = (D == 128);          // dQ^T form (see file comment)
-  static constexpr int STAGES = DQT ? 3 : 2;      // Q_i / dO_i / LSE_i / D_i ring depth
+  static constexpr bool VT = DQT;                 // V_j held in TMEM, dP^T as a TS product
+  static constexpr int STAGES = DQT ? (VT ? 4 : 3) : 2;   // Q_i / dO_i / LSE_i / D_i ring depth
   static constexpr int BM = DQT ? 64 : 128;       // query rows per step
   static constexpr int HALF = BM / 2;             // query columns per compute warpgroup
   static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span of Q/K/V/dO rows (bytes)
@@ -77,10 +78,12 @@ struct BwdCfg {
   // at once):  S^T [0,64) dP^T[0] [64,128) dP^T[1] [128,192) dV [192,320) dK [320,448)
   // dQ^T [448,512).  d <= 64: one dP^T buffer and two dQ slots:
   //   S^T [0,BM) dP^T [BM,2BM) dV, dK (d each) then two dQ slots of d columns.
-  static constexpr int NDPT = DQT ? 2 : 1;           // dP^T buffers
+  static constexpr int NDPT = (DQT && !VT) ? 2 : 1;  // dP^T buffers
   static constexpr int NDQ = DQT ? 1 : 2;            // dQ slots
-  static constexpr int T_ST = 0;
-  static constexpr int T_DPT = BM;                   // dP^T buffer b at T_DPT + b * BM
+  static constexpr int T_V = 0;                      // V_j as a bf16 A operand: D/2 columns
+  static constexpr int V_COLS = VT ? D / 2 : 0;
+  static constexpr int T_ST = V_COLS;
+  static constexpr int T_DPT = T_ST + BM;            // dP^T buffer b at T_DPT + b * BM
   static constexpr int T_DV = T_DPT + NDPT * BM;
   static constexpr int T_DK = T_DV + D;
   static constexpr int T_DQ = T_DK + D;              // NDQ slots of DQ_COLS
@@ -89,12 +92,13 @@ struct BwdCfg {
   // shared memory map (offsets from the 1024-aligned base)
   static constexpr int O_K = 0;
   static constexpr int O_V = O_K + KV_TILE_BYTES;
-  static constexpr int O_Q = O_V + KV_TILE_BYTES;              // STAGES
+  static constexpr int O_Q = O_V + (VT ? 0 : KV_TILE_BYTES);   // STAGES
   static constexpr int O_DO = O_Q + STAGES * Q_TILE_BYTES;      // STAGES
   static constexpr int O_DS = O_DO + STAGES * Q_TILE_BYTES;     // 2 buffers
   // LSE_i * log2 e and D_i rows live in LSLOTS slots (slot n % LSLOTS for step n), each
   // with its own full barrier that the compute warpgroups observe phase by phase.
   static constexpr int LSLOTS = 6;
+  static_assert(LSLOTS >= STAGES, "an LSE slot must outlive the Q stage of its step");
   static constexpr int O_LSE = O_DS + 2 * DS_BYTES;            // LSLOTS x BM floats
   static constexpr int O_DD = O_LSE + LSLOTS * BM * 4;         // LSLOTS x BM floats
   // dQ staging tile for the bulk reduction, [BM query rows][d] fp32.  d = 128: plain
@@ -119,7 +123,8 @@ struct BwdCfg {
   static constexpr int B_DQFULL = B_DSFREE + 2;      // 2
   static constexpr int B_DQEMPTY = B_DQFULL + 2;     // 2
   static constexpr int B_DONE = B_DQEMPTY + 2;
-  static constexpr int NBARS = B_DONE + 1;
+  static constexpr int B_VT = B_DONE + 1;            // V_j written into TMEM
+  static constexpr int NBARS = B_VT + 1;
   static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 16;
 };
 
@@ -131,6 +136,7 @@ struct BwdParams {
   int32_t causal;
   const float* lse;      // [hq, T]
   const float* dd;       // [hq, T]
+  const __nv_bfloat16* v;   // [T, hkv, d] (read directly when V_j lives in TMEM)
   float* dq_acc;         // [T, hq, d]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t cnt = 1;
       // warp-level arrivals: one per compute warp (PT, DS) or drain warp (DQEMPTY)
       if (i == C::B_PT || i == C::B_DS) cnt = 8;
-      if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1) cnt = 4;
+      if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1 || i == C::B_VT) cnt = 4;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -221,10 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 12) {
     // ---------------- producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per step ----------
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE_BYTES);
+      mbar_arrive_expect_tx(bar(C::B_KV), (C::VT ? 1 : 2) * C::KV_TILE_BYTES);
       for (int pn = 0; pn < C::NPANEL; ++pn) {
         tma_load_3d(sbase + C::O_K + pn * C::KV_PANEL_BYTES, &tmK, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
-        tma_load_3d(sbase + C::O_V + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
+        if (!C::VT)
+          tma_load_3d(sbase + C::O_V + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
       }
     }
     // LSE_i * log2(e) and D_i of the next step are loaded into registers one step ahead,
@@ -282,47 +289,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto kmajor_off = [&](int kk, int panel_bytes) {
         return (uint32_t)((kk / C::KSTEPS_PER_PANEL) * panel_bytes + (kk % C::KSTEPS_PER_PANEL) * 32);
       };
+      // Every operand descriptor is a base descriptor (computed once, or once per ring
+      // stage) advanced by a compile-time offset, so issuing one MMA takes a few
+      // instructions; the issue rate of this single thread bounds the tensor core here.
+      const uint64_t k_kmaj = smem_desc(sbase + C::O_K, 16, C::SBO, C::SWZ);               // K, K-major
+      const uint64_t v_kmaj = smem_desc(sbase + C::O_V, 16, C::SBO, C::SWZ);               // V, K-major
+      const uint64_t k_mn = smem_desc(sbase + C::O_K, C::KV_PANEL_BYTES, C::SBO, C::SWZ);  // K^T operand
+      const uint64_t q_kmaj = smem_desc(sbase + C::O_Q, 16, C::SBO, C::SWZ);
+      const uint64_t do_kmaj = smem_desc(sbase + C::O_DO, 16, C::SBO, C::SWZ);
+      const uint64_t q_mn = smem_desc(sbase + C::O_Q, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
+      const uint64_t do_mn = smem_desc(sbase + C::O_DO, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
+      const uint64_t ds_desc = smem_desc(sbase + C::O_DS, C::DS_PANEL_BYTES, 1024, 2u);
+      auto stage = [&](uint64_t base, int s) { return desc_advance(base, (uint32_t)s * C::Q_TILE_BYTES); };
       // X_tile (128 keys) times Y_i^T (BM rows), both K-major over d
-      auto issue_sdp = [&](uint32_t x_off, uint32_t y_off, uint32_t d_col) {
+      auto issue_sdp = [&](uint64_t x, uint64_t y, uint32_t d_col) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = smem_desc(sbase + x_off + kmajor_off(kk, C::KV_PANEL_BYTES), 16, C::SBO, C::SWZ);
-          const uint64_t bd = smem_desc(sbase + y_off + kmajor_off(kk, C::Q_PANEL_BYTES), 16, C::SBO, C::SWZ);
-          mma_ss(tmem + d_col, a, bd, id_sdp, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + d_col, desc_advance(x, kmajor_off(kk, C::KV_PANEL_BYTES)),
+                 desc_advance(y, kmajor_off(kk, C::Q_PANEL_BYTES)), id_sdp, kk > 0 ? 1u : 0u);
       };
       // D[128 keys x d] += A^T(TMEM, bf16 over BM queries) * Y_i (BM x d, MN-major).
       // Each compute warpgroup packs its half of the queries into the first columns of
       // its own half of the fp32 region, so queries [h*HALF, (h+1)*HALF) sit at columns
       // h*HALF + (q - h*HALF)/2.
-      auto issue_grad = [&](uint32_t a_col, uint32_t y_off, uint32_t d_col, bool acc) {
+      auto issue_grad = [&](uint32_t a_col, uint64_t y, uint32_t d_col, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const int qb = kk * 16;
           const int hh = qb / HALF;
           const uint32_t col = a_col + hh * HALF + (qb - hh * HALF) / 2;
-          const uint64_t bd = smem_desc(sbase + y_off + kk * 16 * C::SW, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
-          mma_ts(tmem + d_col, tmem + col, bd, id_grad, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + d_col, tmem + col, desc_advance(y, kk * 16 * C::SW), id_grad, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      // dP^T = V_j dO_i^T: from shared memory, or with V_j (A) read out of TMEM
+      auto issue_dpt = [&](uint64_t y, uint32_t d_col) {
+        if (C::VT) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ts(tmem + d_col, tmem + C::T_V + kk * 8, desc_advance(y, kmajor_off(kk, C::Q_PANEL_BYTES)), id_sdp,
+                   kk > 0 ? 1u : 0u);
+        } else {
+          issue_sdp(v_kmaj, y, d_col);
         }
       };
       auto issue_dq = [&](int dsbuf, uint32_t d_col) {
-        const uint32_t ds = sbase + C::O_DS + dsbuf * C::DS_BYTES;
+        const uint64_t ds = desc_advance(ds_desc, (uint32_t)dsbuf * C::DS_BYTES);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t kdesc = smem_desc(sbase + C::O_K + kk * 16 * C::SW, C::KV_PANEL_BYTES, C::SBO, C::SWZ);
-          const uint64_t sdesc = smem_desc(ds + kk * 16 * 128, C::DS_PANEL_BYTES, 1024, 2u);
+          const uint64_t kd = desc_advance(k_mn, kk * 16 * C::SW);
+          const uint64_t sd = desc_advance(ds, kk * 16 * 128);
           if (C::DQT)
-            mma_ss(tmem + d_col, kdesc, sdesc, id_dq, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + d_col, kd, sd, id_dq, kk > 0 ? 1u : 0u);
           else
-            mma_ss(tmem + d_col, sdesc, kdesc, id_dq, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + d_col, sd, kd, id_dq, kk > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag) && mbar_wait(bar(C::B_QFULL), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_sdp(C::O_K, C::O_Q, C::T_ST);
+        issue_sdp(k_kmaj, q_kmaj, C::T_ST);
         mma_commit(bar(C::B_ST));
-        issue_sdp(C::O_V, C::O_DO, C::T_DPT);
+        ok = !C::VT || mbar_wait(bar(C::B_VT), 0, abort_flag);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dpt(do_kmaj, C::T_DPT);
         mma_commit(bar(C::B_DPT));
       }
       // Order per step n (dP^T buffer db = n & 1 when NDPT == 2, else 0):
@@ -337,33 +368,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int db1 = C::NDPT == 2 ? (b2 ^ 1) : 0;
         const int qslot = C::NDQ == 2 ? b2 : 0;
         const uint32_t qpar = C::NDQ == 2 ? (((n >> 1) & 1) ^ 1) : (uint32_t)((n & 1) ^ 1);
-        const uint32_t q_off = C::O_Q + s * C::Q_TILE_BYTES;
-        const uint32_t do_off = C::O_DO + s * C::Q_TILE_BYTES;
         const bool more = n + 1 < n_steps;
         if (!mbar_wait(bar(C::B_PT), n & 1, abort_flag)) break;
         tc_fence_after();
-        issue_grad(C::T_ST, do_off, C::T_DV, n > 0);                  // dV += P^T dO
+        issue_grad(C::T_ST, stage(do_mn, s), C::T_DV, n > 0);                 // dV += P^T dO
         if (more) {
           if (!mbar_wait(bar(C::B_QFULL + s1), ((n + 1) / C::STAGES) & 1, abort_flag)) break;
           tc_fence_after();
-          issue_sdp(C::O_K, C::O_Q + s1 * C::Q_TILE_BYTES, C::T_ST);   // S^T for the next step
+          issue_sdp(k_kmaj, stage(q_kmaj, s1), C::T_ST);                      // S^T for the next step
           mma_commit(bar(C::B_ST));
           if (C::NDPT == 2) {
-            issue_sdp(C::O_V, C::O_DO + s1 * C::Q_TILE_BYTES, C::T_DPT + db1 * BM);   // dP^T(n+1)
+            issue_dpt(stage(do_kmaj, s1), C::T_DPT + db1 * BM);               // dP^T(n+1)
             mma_commit(bar(C::B_DPT + db1));
           }
         }
         if (!mbar_wait(bar(C::B_DS), n & 1, abort_flag)) break;
         tc_fence_after();
-        issue_grad(C::T_DPT + db * BM, q_off, C::T_DK, n > 0);        // dK += dS^T Q
+        issue_grad(C::T_DPT + db * BM, stage(q_mn, s), C::T_DK, n > 0);       // dK += dS^T Q
         mma_commit(bar(C::B_QEMPTY + s));
         if (!mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) break;
         tc_fence_after();
-        issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                    // dQ_i partial
+        issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                           // dQ_i partial
         mma_commit(bar(C::B_DQFULL + qslot));
         mma_commit(bar(C::B_DSFREE + b2));
         if (C::NDPT == 1 && more) {
-          issue_sdp(C::O_V, C::O_DO + s1 * C::Q_TILE_BYTES, C::T_DPT);  // dP^T for the next step
+          issue_dpt(stage(do_kmaj, s1), C::T_DPT);                            // dP^T for the next step
           mma_commit(bar(C::B_DPT));
         }
       }
@@ -378,6 +407,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = half * HALF;                   // first query column of this thread
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     const float sl2 = p.scale_log2;
+    if (C::VT && half == 0) {
+      // V_j row kr, bf16 pairs as they lie in memory (element 2c in the low half of column
+      // c), is the A operand of dP^T; rows past the sequence are zero.
+      const uint4* vrow = reinterpret_cast<const uint4*>(p.v + ((size_t)(seq_start + kj) * p.hkv + g) * D);
+#pragma unroll
+      for (int cb = 0; cb < C::V_COLS; cb += 32) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 x = kj < len ? vrow[cb / 4 + e] : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * e] = x.x;
+          w[4 * e + 1] = x.y;
+          w[4 * e + 2] = x.z;
+          w[4 * e + 3] = x.w;
+        }
+        tmem_st32(trow + C::T_V + cb, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_VT));
+    }
     bool ok = true;
     for (int n = 0; n < n_steps; ++n) {
       const int ls = n % C::LSLOTS;
@@ -514,6 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lane = feature c, registers = the BM query rows of this step.  The partial is
         // transposed into a [BM][d] fp32 staging tile and added into the accumulator by
         // one bulk tensor reduction (query rows past the sequence carry exact zeros).
+        // (Per-lane red.global.add from registers would skip shared memory but measured
+        // well below the bulk reduction's throughput.)
         const int c = lane_base + lane;
         float* stg = reinterpret_cast<float*>(smem + C::O_STG);
 #pragma unroll
@@ -676,6 +729,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   p.causal = pb.causal;
   p.lse = lse;
   p.dd = dd;
+  p.v = static_cast<const __nv_bfloat16*>(v);
   p.dq_acc = dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

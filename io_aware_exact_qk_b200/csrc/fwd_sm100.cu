@@ -228,23 +228,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kRows, kKeys, false, false);  // Q, K both K-major
       const uint32_t idesc_pv = idesc_bf16_f32(kRows, D, false, true);       // V is MN-major (d contiguous)
+      // Operand descriptors: bases computed once, advanced by compile-time offsets per
+      // MMA (and by the tile/stage index per call), so one MMA issues in a few
+      // instructions -- this single thread's issue rate bounds the tensor core.
+      const uint64_t q_desc = smem_desc(sQ, 16, C::SBO, C::SWZ);
+      const uint64_t k_desc = smem_desc(sK, 16, C::SBO, C::SWZ);
+      const uint64_t v_desc = smem_desc(sV, C::PANEL_BYTES, C::SBO, C::SWZ);
       auto issue_qk = [&](int t, int s) {
         const uint32_t d_tmem = tmem + t * kKeys;
+        const uint64_t a0 = desc_advance(q_desc, (uint32_t)t * C::TILE_BYTES);
+        const uint64_t b0 = desc_advance(k_desc, (uint32_t)s * C::TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / C::KSTEPS_PER_PANEL) * C::PANEL_BYTES + (kk % C::KSTEPS_PER_PANEL) * 32;
-          const uint64_t a = smem_desc(sQ + t * C::TILE_BYTES + off, 16, C::SBO, C::SWZ);
-          const uint64_t bd = smem_desc(sK + s * C::TILE_BYTES + off, 16, C::SBO, C::SWZ);
-          mma_ss(d_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss(d_tmem, desc_advance(a0, off), desc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int s, bool accumulate) {
         const uint32_t d_tmem = tmem + 2 * kKeys + t * D;
+        const uint64_t b0 = desc_advance(v_desc, (uint32_t)s * C::TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           const uint32_t a_tmem = tmem + t * kKeys + kk * 8;   // 16 bf16 keys = 8 packed columns
-          const uint64_t bd = smem_desc(sV + s * C::TILE_BYTES + kk * 16 * C::SW, C::PANEL_BYTES, C::SBO, C::SWZ);
-          mma_ts(d_tmem, a_tmem, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem, desc_advance(b0, kk * 16 * C::SW), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       uint32_t kv = 0, qi = 0;
