@@ -20,6 +20,14 @@ for causal masks, max-value stability and packed variable-length sequences; the
   gqa8k     B=2,  Hq=32, Hkv=8, N=8192, d=128, causal   (+ x30 stability variant)
   varlen16  16 sequences, lengths U{64..4096}, H=16, d=128, causal
   long32k   B=1,  H=16, N=32768, d=128, causal
+
+Decoding-shaped workloads (the tutorial's FlashDecoding case, "one query against a long
+KV"): sequence b has Lq_b query rows (the newest tokens) and Lk_b cached keys; Q is
+[sum Lq, Hq, d], K and V are [sum Lk, Hkv, d], drawn in the order (lengths, Q, K, V):
+
+  decode8k      16 sequences, Lq=1, Lk=8192,          Hq=32, Hkv=8, d=128
+  decode_var    16 sequences, Lq=1, Lk ~ U{64..32768}, Hq=32, Hkv=8, d=128
+  decode_spec4  16 sequences, Lq=4 (causal), Lk=4096,  Hq=32, Hkv=8, d=128
 """
 from __future__ import annotations
 
@@ -142,3 +150,85 @@ def make_inputs(w: Workload, dtype: torch.dtype = torch.bfloat16, with_grad: boo
         q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
         do = do.to(dtype) if do is not None else None
     return q, k, v, do, w.cu_seqlens()
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    q_lens: tuple           # query rows per sequence (the newest positions)
+    k_lens: tuple           # keys per sequence
+    hq: int
+    hkv: int
+    d: int
+    causal: bool
+    seed: int
+    random_k: Optional[tuple] = None   # (lo, hi): k_lens drawn from the seed stream first
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def batch(self) -> int:
+        return len(self.k_lens)
+
+    @property
+    def total_q(self) -> int:
+        return sum(self.q_lens)
+
+    @property
+    def total_k(self) -> int:
+        return sum(self.k_lens)
+
+    @property
+    def max_k(self) -> int:
+        return max(self.k_lens) if self.k_lens else 0
+
+    def cu_q(self) -> torch.Tensor:
+        return torch.tensor([0] + [sum(self.q_lens[:i + 1]) for i in range(len(self.q_lens))], dtype=torch.int32)
+
+    def cu_k(self) -> torch.Tensor:
+        return torch.tensor([0] + [sum(self.k_lens[:i + 1]) for i in range(len(self.k_lens))], dtype=torch.int32)
+
+    def kv_bytes(self) -> int:
+        """Bytes of K and V (bf16) that any exact decode must read once."""
+        return 2 * self.total_k * self.hkv * self.d * 2
+
+    def hbm_bytes(self) -> int:
+        """Algorithmic HBM traffic: K, V read, Q read, O written (bf16), LSE written (fp32)."""
+        return self.kv_bytes() + 2 * self.total_q * self.hq * self.d * 2 + 4 * self.total_q * self.hq
+
+
+def _decode_lengths(seed: int, count: int, lo: int, hi: int) -> tuple:
+    g = torch.Generator().manual_seed(seed)
+    return tuple(int(x) for x in torch.randint(lo, hi + 1, (count,), generator=g))
+
+
+def decode8k() -> DecodeWorkload:
+    return DecodeWorkload("decode8k", (1,) * 16, (8192,) * 16, 32, 8, 128, False, seed=1101)
+
+
+def decode_var() -> DecodeWorkload:
+    return DecodeWorkload("decode_var", (1,) * 16, _decode_lengths(1102, 16, 64, 32768), 32, 8, 128, False,
+                          seed=1102, random_k=(64, 32768))
+
+
+def decode_spec4() -> DecodeWorkload:
+    return DecodeWorkload("decode_spec4", (4,) * 16, (4096,) * 16, 32, 8, 128, True, seed=1103)
+
+
+def decode_custom(name, q_lens, k_lens, hq, hkv, d, causal, seed) -> DecodeWorkload:
+    return DecodeWorkload(name, tuple(int(x) for x in q_lens), tuple(int(x) for x in k_lens), hq, hkv, d, causal, seed)
+
+
+def make_decode_inputs(w: DecodeWorkload, dtype: torch.dtype = torch.bfloat16):
+    """Seeded CPU tensors q [sum Lq,Hq,d], k, v [sum Lk,Hkv,d], cu_q, cu_k (int32)."""
+    g = torch.Generator().manual_seed(w.seed)
+    if w.random_k is not None:
+        torch.randint(w.random_k[0], w.random_k[1] + 1, (len(w.k_lens),), generator=g)   # the lengths came first
+    q = torch.randn(w.total_q, w.hq, w.d, generator=g, dtype=torch.float32)
+    k = torch.randn(w.total_k, w.hkv, w.d, generator=g, dtype=torch.float32)
+    v = torch.randn(w.total_k, w.hkv, w.d, generator=g, dtype=torch.float32)
+    if dtype != torch.float32:
+        q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
+    return q, k, v, w.cu_q(), w.cu_k()

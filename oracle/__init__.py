@@ -41,6 +41,7 @@ def _bind(lib):
                                        up, up, dp, dp, dp, dp, dp, dp, dp, i32]
     lib.oracle_attn_bwd_ex.restype = ctypes.c_int
     lib.oracle_attn_probs.argtypes = [dp, dp, i32, i32, f64, i32, dp, dp]
+    lib.oracle_attn_fwd_cross.argtypes = [dp, dp, dp, ip, ip, i32, i32, i32, i32, f64, i32, dp, dp, i32]
     lib.oracle_attn_probs.restype = ctypes.c_int
     _lib = lib
 
@@ -114,6 +115,29 @@ def attn_fwd(q, k, v, cu_seqlens=None, scale=None, causal=False, rows=None, thre
                                  _ptr(o), _ptr(lse), threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
+    return o, lse
+
+
+def attn_fwd_cross(q, k, v, cu_q, cu_k, scale=None, causal=False, threads=None):
+    """Decoding-shaped forward: sequence b has cu_q[b+1]-cu_q[b] query rows (the last
+    positions of the sequence) and cu_k[b+1]-cu_k[b] keys.  O [Tq,Hq,d], LSE [Hq,Tq]
+    (float64); under ``causal`` query row i sees keys j <= Lk - Lq + i."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Tq, hq, d = q.shape
+    hkv = k.shape[1]
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    if len(cq) != len(ck) or cq[-1] != Tq or ck[-1] != k.shape[0]:
+        raise ValueError("cu_q / cu_k do not match the tensors")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.full((Tq, hq, d), np.nan)
+    lse = np.full((hq, Tq), np.nan)
+    rc = _load().oracle_attn_fwd_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(cq, ctypes.c_int32), _ptr(ck, ctypes.c_int32),
+                                       len(cq) - 1, hq, hkv, d, float(scale), int(bool(causal)), _ptr(o), _ptr(lse),
+                                       threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_cross failed with code {rc}")
     return o, lse
 
 

@@ -325,6 +325,102 @@ static int check_args(const int32_t *cu, int32_t nseq, int32_t hq, int32_t hkv, 
     return ORACLE_OK;
 }
 
+/* ---- decoding forward: fewer query rows than keys ----------------------------------
+ * "FlashAttention 与高效注意力内核" tutorial, section "FlashAttention 变体族谱": the decode
+ * variant (FlashDecoding) serves "one query against a long KV".  What it computes is the
+ * same three steps as above; only the shapes differ.  Sequence b has
+ * Lq = cu_q[b+1] - cu_q[b] query rows and Lk = cu_k[b+1] - cu_k[b] keys, and the query
+ * rows are the LAST Lq positions of the sequence (the tokens being decoded), so under the
+ * causal mask query row i (0-based inside its sequence) sees keys j <= Lk - Lq + i, none
+ * when that is negative.  With Lq = Lk this is the self-attention mask above.
+ * Layouts: q, o [Tq, hq, d]; k, v [Tk, hkv, d]; lse [hq, Tq] with Tq = cu_q[nseq]. */
+typedef struct {
+    problem P;                  /* q, k, v, hq, hkv, d, scale, causal, o, lse */
+    const int32_t *cu_q, *cu_k;
+    int32_t nseq;
+    int64_t tq;
+    int64_t next, nitems;       /* items: (sequence, query head) */
+    pthread_mutex_t lock;
+    int failed;
+} cross_work;
+
+static int cross_visible(int i, int lq, int lk, int causal)
+{
+    if (!causal) return lk;
+    const int v = lk - lq + i + 1;
+    return v < 0 ? 0 : (v > lk ? lk : v);
+}
+
+static void *cross_worker(void *arg)
+{
+    cross_work *W = (cross_work *)arg;
+    problem *P = &W->P;
+    int64_t maxk = 1;
+    for (int b = 0; b < W->nseq; ++b) {
+        const int64_t n = W->cu_k[b + 1] - W->cu_k[b];
+        if (n > maxk) maxk = n;
+    }
+    double *s = (double *)malloc((size_t)maxk * sizeof(double));
+    double *p = (double *)malloc((size_t)maxk * sizeof(double));
+    if (!s || !p) {
+        pthread_mutex_lock(&W->lock); W->failed = 1; pthread_mutex_unlock(&W->lock);
+        free(s); free(p);
+        return NULL;
+    }
+    for (;;) {
+        pthread_mutex_lock(&W->lock);
+        const int64_t it = W->next++;
+        pthread_mutex_unlock(&W->lock);
+        if (it >= W->nitems) break;
+        const int b = (int)(it / P->hq);
+        const int h = (int)(it % P->hq);
+        const int64_t q0 = W->cu_q[b], k0 = W->cu_k[b];
+        const int lq = (int)(W->cu_q[b + 1] - q0), lk = (int)(W->cu_k[b + 1] - k0);
+        for (int i = 0; i < lq; ++i) {
+            const int64_t row = q0 + i;
+            const int vis = cross_visible(i, lq, lk, P->causal);
+            score_row(P, row, k0, lk, vis, h, s);
+            const double lse = softmax_row(s, lk, p);
+            output_row(P, k0, lk, h, p, P->o + (row * P->hq + h) * P->d);
+            P->lse[(int64_t)h * W->tq + row] = lse;
+        }
+    }
+    free(s);
+    free(p);
+    return NULL;
+}
+
+int oracle_attn_fwd_cross(const double *q, const double *k, const double *v,
+                          const int32_t *cu_q, const int32_t *cu_k, int32_t nseq,
+                          int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                          double *o, double *lse, int32_t nthreads)
+{
+    int rc = check_args(cu_q, nseq, hq, hkv, d);
+    if (rc) return rc;
+    rc = check_args(cu_k, nseq, hq, hkv, d);
+    if (rc) return rc;
+    cross_work W;
+    memset(&W, 0, sizeof W);
+    W.P.q = q; W.P.k = k; W.P.v = v; W.P.hq = hq; W.P.hkv = hkv; W.P.d = d;
+    W.P.scale = scale; W.P.causal = causal; W.P.o = o; W.P.lse = lse;
+    W.cu_q = cu_q; W.cu_k = cu_k; W.nseq = nseq; W.tq = cu_q[nseq];
+    W.nitems = (int64_t)nseq * hq;
+    pthread_mutex_init(&W.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    pthread_t *tid = (pthread_t *)malloc((size_t)nthreads * sizeof(pthread_t));
+    int started = 0;
+    if (tid) {
+        for (; started < nthreads; ++started)
+            if (pthread_create(&tid[started], NULL, cross_worker, &W) != 0) break;
+    }
+    if (started == 0) cross_worker(&W);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    free(tid);
+    pthread_mutex_destroy(&W.lock);
+    return W.failed ? ORACLE_NO_MEM : ORACLE_OK;
+}
+
 /* Forward: o [T,hq,d], lse [hq,T].  row_sel (optional, [T]) restricts which rows are
  * written; other entries of o and lse are left untouched. */
 int oracle_attn_fwd(const double *q, const double *k, const double *v,

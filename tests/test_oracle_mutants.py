@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_decode as dpins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
 
@@ -31,6 +32,11 @@ MUTANTS = {
                           "if (lse_in) lse[(int64_t)h * T + t] = lse[(int64_t)h * T + t];"),
     "given O ignored for D": ("dd[(int64_t)h * T + t] = dsum;", "(void)dsum;"),
     "score mask boundary off by one": ("if (j >= vis) { s[j] = -INFINITY; continue; }", "if (j > vis) { s[j] = -INFINITY; continue; }"),
+    "decode causal mask aligned top-left": ("const int v = lk - lq + i + 1;", "const int v = i + 1;"),
+    "decode LSE stored to the sequence's first row": ("P->lse[(int64_t)h * W->tq + row] = lse;",
+                                                      "P->lse[(int64_t)h * W->tq + q0] = lse;"),
+    "decode keys addressed by the query offsets": ("score_row(P, row, k0, lk, vis, h, s);",
+                                                   "score_row(P, row, q0, lk, vis, h, s);"),
     "value row from the wrong key": ("const double *vj = P->v + ((key0 + j) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]",
                                      "const double *vj = P->v + ((key0 + (n - 1 - j)) * P->hkv + g) * d;\n        for (int c = 0; c < d; ++c) oi[c]"),
 }
@@ -49,6 +55,9 @@ def _battery():
         lambda: pins.test_gradient_invariants(False),
         lambda: pins.test_given_lse_shift_scales_gradients_exactly(),
         lambda: pins.test_given_o_changes_dq_by_closed_form(),
+        lambda: dpins.test_cross_matches_brute_force(([1, 3], [2, 6]), True),
+        lambda: dpins.test_cross_matches_brute_force(([2, 3], [7, 3]), False),
+        lambda: dpins.test_cross_zero_queries_average_the_visible_values(),
     ]
     for c in checks:
         try:
