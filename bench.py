@@ -17,6 +17,7 @@ write) between timed steps, per-kernel times from the library's own launch event
 sample of the same workload, on rank 0 only.
 """
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -336,6 +337,174 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------------------
+# Decoding workloads (split-KV forward): HBM-bound, reported in GB/s of algorithmic traffic
+# ---------------------------------------------------------------------------------------
+DECODE_METRIC = "split-KV decode forward: algorithmic HBM GB/s (K, V, Q read once, O, LSE written) on 1 B200"
+DECODE_WORKLOADS = {"decode8k": W.decode8k, "decode_var": W.decode_var, "decode_spec4": W.decode_spec4}
+DECODE_DATA = ("synthetic: Q, K, V iid N(0,1) drawn in fp32 from a seeded torch CPU generator (decode_var: key "
+               "lengths drawn first from the same generator), rounded to bf16")
+
+
+def decode_config(n_gpus):
+    w = DECODE_WORKLOADS[WORKLOAD]()
+    return {"workload": f"{WORKLOAD}: {w.batch} sequences, Lq={sorted(set(w.q_lens))}, Lk max {w.max_k} "
+                        f"(total {w.total_k}), Hq={w.hq} Hkv={w.hkv} d={w.d} bf16, "
+                        + ("causal" if w.causal else "non-causal"),
+            "global_batch": w.batch * n_gpus, "kv_bytes": w.kv_bytes(), "hbm_bytes_per_step": w.hbm_bytes(),
+            "l2": "inputs larger than L2 (K/V of 268-979 MB against 126 MB), no flush between steps (a 256 MiB "
+                  "write would leave dirty lines whose write-back competes with the reads)",
+            "parallelism": f"replicas x{n_gpus}"}
+
+
+def decode_oracle_sample(budget_s):
+    """Oracle decode forward on whole sequences (all heads) until the budget is spent.
+    Returns (algorithmic bytes of the sequences done, seconds, sequences, threads)."""
+    import oracle
+    w = DECODE_WORKLOADS[WORKLOAD]()
+    if "decode" not in _ORACLE_CACHE:
+        _ORACLE_CACHE["decode"] = W.make_decode_inputs(w)
+    q, k, v, cu_q, cu_k = _ORACLE_CACHE["decode"]
+    threads = oracle.default_threads()
+    nbytes, secs, done = 0, 0.0, 0
+    for b in range(w.batch):
+        if secs >= budget_s and done > 0:
+            break
+        qs, ks, vs = q[cu_q[b]:cu_q[b + 1]], k[cu_k[b]:cu_k[b + 1]], v[cu_k[b]:cu_k[b + 1]]
+        lq, lk = int(cu_q[b + 1] - cu_q[b]), int(cu_k[b + 1] - cu_k[b])
+        t0 = time.perf_counter()
+        oracle.attn_fwd_cross(qs, ks, vs, [0, lq], [0, lk], scale=w.scale, causal=w.causal, threads=threads)
+        secs += time.perf_counter() - t0
+        nbytes += 2 * lk * w.hkv * w.d * 2 + 2 * lq * w.hq * w.d * 2 + 4 * lq * w.hq
+        done += 1
+    return nbytes, secs, done, threads
+
+
+def run_reference_decode(args, rank, world):
+    if rank != 0:
+        return
+    decode_oracle_sample(0.0)
+    nbytes = secs = 0.0
+    threads = 1
+    for _ in range(args.steps):
+        b, s_, _, threads = decode_oracle_sample(0.0)   # one whole sequence per step
+        nbytes += b
+        secs += s_
+    value = nbytes / secs / 1e9
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DECODE_DATA,
+            "config": decode_config(world),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"fp64 CPU oracle, sequence 0 of {WORKLOAD} (all heads) per step"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_decode(args, rank, world, local_rank):
+    import io_aware_exact_qk_b200 as attn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    attn.load_library()
+    w = DECODE_WORKLOADS[WORKLOAD]()
+    w = dataclasses.replace(w, seed=w.seed + rank)
+    q, k, v, cu_q, cu_k = W.make_decode_inputs(w)
+    qd, kd, vd, cqd, ckd = (t.to(dev) for t in (q, k, v, cu_q, cu_k))
+    mq = max(w.q_lens)
+    ws_bytes = attn.decode_workspace_size(qd, kd, cqd, ckd, mq, w.max_k)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty(w.hq, w.total_q, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.attn_fwd_decode(qd, kd, vd, cqd, ckd, mq, w.max_k, scale=w.scale, causal=w.causal, o=o, lse=lse,
+                             workspace=ws)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    attn.attn_get_device_error()
+    barrier()
+    attn.attn_profile_collect()
+    attn.attn_profile_enable(True)
+    launches0 = attn.attn_launch_count()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        for s_, e_ in events:
+            s_.record(stream)
+            step()
+            e_.record(stream)
+        barrier()
+    attn.attn_profile_enable(False)
+    launches = attn.attn_launch_count() - launches0
+    per_kernel = attn.attn_profile_collect()
+    attn.attn_get_device_error()
+    total_ms = sum(s_.elapsed_time(e_) for s_, e_ in events)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = world * w.hbm_bytes() * args.steps / (total_ms / 1e3) / 1e9
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"quick": True, "value": value, "unit": "GB/s", "ms_per_step": total_ms / args.steps,
+                              "kernels": {k_: list(v_) for k_, v_ in per_kernel.items()}, "gpu_launches": launches}))
+        return
+    # end to end: the caller's Q/K/V in pinned host memory, O and LSE back to the host
+    hq_, hk_, hv_ = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    ho, hl = torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(lse.shape).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        qd.copy_(hq_, non_blocking=True)
+        kd.copy_(hk_, non_blocking=True)
+        vd.copy_(hv_, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    attn.attn_get_device_error()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * w.hbm_bytes() * args.steps / (float(t.item()) / 1e3) / 1e9
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    dom = max(per_kernel, key=lambda n_: per_kernel[n_][0])
+    dom_ms, dom_n = per_kernel[dom]
+    dom_bytes = w.hbm_bytes() if dom.startswith("decode_bf16") else 0
+    achieved = dom_bytes * args.steps / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks['source']} HBM copy bandwidth",
+                "bytes_per_launch": dom_bytes * args.steps / dom_n, "mean_launch_ms": dom_ms / dom_n}
+    breakdown = {k_: {"launches": n_, "total_ms": ms, "share": ms / sum(x[0] for x in per_kernel.values())}
+                 for k_, (ms, n_) in sorted(per_kernel.items())}
+    cpu = None
+    if world == 1:
+        b, s_, done, threads = decode_oracle_sample(12.0)
+        cpu = {"value": b / s_ / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"fp64 CPU oracle, {done} whole sequence(s) of {WORKLOAD} (all heads), {s_:.1f} s"}
+    line = {"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DECODE_DATA, "config": decode_config(world),
+            "pct_of_peak": value / peaks["hbm_gbs"], "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "clocks": clocks.summary(), "kernels": breakdown}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,7 +512,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha2k",
-                    help="mha2k (the metric's configuration), sweep_d<d>_n<N>, gqa8k, varlen16 or long32k")
+                    help="mha2k (the metric's configuration), sweep_d<d>_n<N>, gqa8k, varlen16, long32k; "
+                         "or a split-KV decode workload: decode8k, decode_var, decode_spec4")
     ap.add_argument("--quick", action="store_true",
                     help="device timing only: skip the end-to-end loop and the CPU baseline (profiling runs)")
     args = ap.parse_args()
@@ -356,8 +526,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    decode = WORKLOAD in DECODE_WORKLOADS
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        (run_reference_decode if decode else run_reference)(args, rank, world)
         return
     if world > 1:
         import datetime
@@ -365,7 +536,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        (run_decode if decode else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

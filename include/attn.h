@@ -123,6 +123,45 @@ attn_status attn_bwd_noalloc(const void *q, const void *k, const void *v,
                              float scale, int32_t causal, int32_t dtype,
                              void *dq, void *dk, void *dv, void *stream);
 
+/* Decoding forward (split-KV).  The tutorial's FlashDecoding variant (section
+ * "FlashAttention 变体族谱": one query against a long KV, the KV cut into blocks whose
+ * partial results are computed in parallel and then reduced; section "变体选择场景":
+ * decoding is bandwidth-bound).  The result is the forward's definition for sequences whose
+ * query rows are the newest positions of a longer key/value sequence: sequence b has
+ * Lq_b query rows and Lk_b keys, and under `causal` query row t (0-based) sees keys
+ * j <= Lk_b - Lq_b + t (bottom-right alignment; with Lq_b = Lk_b this is attn_fwd's mask).
+ *     q, o   [total_q, hq, d]  bf16        k, v  [total_k, hkv, d]  bf16
+ *     lse    [hq, total_q]     float32 (natural log; -inf and O = 0 for a row with no key)
+ * Shapes: batch mode passes cu_seqlens_q = cu_seqlens_k = NULL and fixed seqlen_q /
+ * seqlen_k (total_q = batch * seqlen_q, total_k = batch * seqlen_k); varlen mode passes
+ * both DEVICE prefix-sum arrays (int32[batch + 1]) and bounds max_seqlen_q / max_seqlen_k
+ * (a sequence exceeding them is reported by attn_get_device_error as
+ * ATTN_ERR_INVALID_ARG).  The hq / hkv query heads of a KV head and their newest
+ * max_seqlen_q tokens share one 128-row tile: (hq / hkv) * max_seqlen_q <= 128, else
+ * ATTN_ERR_UNSUPPORTED.  d in {32, 64, 128}; bf16 only.
+ * num_splits: key splits per (sequence, KV head); 0 lets the library choose from the
+ * shape and the SM count.  With more than one split the partial results go through the
+ * caller's workspace (attn_fwd_decode_workspace_size() bytes, same num_splits) and a
+ * combine kernel; with one split the workspace is unused (may be NULL, size 0). */
+attn_status attn_fwd_decode(const void *q, const void *k, const void *v,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            int32_t batch, int32_t seqlen_q, int32_t seqlen_k,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k,
+                            int32_t total_q, int32_t total_k,
+                            int32_t hq, int32_t hkv, int32_t d,
+                            float scale, int32_t causal, int32_t num_splits,
+                            void *o, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes attn_fwd_decode needs (0 when one split suffices) for the same shape
+ * arguments; varlen = 1 when cu_seqlens_q / cu_seqlens_k will be passed (batch mode: the
+ * max_seqlen values are seqlen_q / seqlen_k).  With num_splits == 0 the split count, and so
+ * the size, depends on the current device's SM count: query it on the device that runs
+ * the call. */
+size_t attn_fwd_decode_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                      int32_t total_q, int32_t total_k, int32_t hq, int32_t hkv,
+                                      int32_t d, int32_t varlen, int32_t num_splits);
+
 /* Workspace bytes attn_fwd / attn_bwd need for these shape arguments (0 = none). */
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,
                                int32_t hq, int32_t hkv, int32_t d, int32_t dtype);

@@ -71,6 +71,10 @@ def load_library():
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                      vp, vp, vp, vp]
     lib.attn_bwd_noalloc.restype = ctypes.c_int
+    lib.attn_fwd_decode.argtypes = [vp, vp, vp, vp, vp] + [i32] * 10 + [f32, i32, i32, vp, vp, vp, sz, vp]
+    lib.attn_fwd_decode.restype = ctypes.c_int
+    lib.attn_fwd_decode_workspace_size.argtypes = [i32] * 10
+    lib.attn_fwd_decode_workspace_size.restype = sz
     lib.attn_launch_count.argtypes = []
     lib.attn_launch_count.restype = ctypes.c_int64
     _lib = lib
@@ -182,6 +186,54 @@ def attn_bwd_noalloc(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scal
                                 seqlen, ms, T, hq, hkv, d, float(scale), int(bool(causal)), _dtype_code(q),
                                 _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))
     return dq, dk, dv
+
+
+def _decode_shape(q, k, cu_q, cu_k, max_seqlen_q, max_seqlen_k, batch):
+    Tq, hq, d = q.shape
+    Tk, hkv = k.shape[0], k.shape[1]
+    if (cu_q is None) != (cu_k is None):
+        raise ValueError("give both cu_seqlens_q and cu_seqlens_k, or neither")
+    if cu_q is None:
+        if batch is None:
+            raise ValueError("batch mode needs batch=")
+        sq, sk = Tq // batch if batch else 0, Tk // batch if batch else 0
+        return batch, sq, sk, sq, sk, Tq, Tk, hq, hkv, d
+    if max_seqlen_q is None or max_seqlen_k is None:
+        raise ValueError("varlen mode needs max_seqlen_q= and max_seqlen_k=")
+    return len(cu_q) - 1, 0, 0, int(max_seqlen_q), int(max_seqlen_k), Tq, Tk, hq, hkv, d
+
+
+def decode_workspace_size(q, k, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
+                          batch=None, num_splits=0):
+    b, _, _, mq, mk, Tq, Tk, hq, hkv, d = _decode_shape(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                                        max_seqlen_k, batch)
+    return int(load_library().attn_fwd_decode_workspace_size(b, mq, mk, Tq, Tk, hq, hkv, d,
+                                                             int(cu_seqlens_q is not None), int(num_splits)))
+
+
+def attn_fwd_decode(q, k, v, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
+                    scale=None, causal=False, batch=None, num_splits=0, o=None, lse=None, workspace=None,
+                    stream=None):
+    """Split-KV decoding forward: sequence b has Lq query rows (the newest positions) and Lk
+    keys.  Returns (o [Tq,Hq,d] bf16, lse [Hq,Tq] fp32)."""
+    lib = load_library()
+    b, sq, sk, mq, mk, Tq, Tk, hq, hkv, d = _decode_shape(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                                          max_seqlen_k, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(hq, Tq, dtype=torch.float32, device=q.device)
+    ws = int(lib.attn_fwd_decode_workspace_size(b, mq, mk, Tq, Tk, hq, hkv, d, int(cu_seqlens_q is not None),
+                                                int(num_splits)))
+    if ws and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _check(lib.attn_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), b, sq, sk, mq, mk,
+                               Tq, Tk, hq, hkv, d, float(scale), int(bool(causal)), int(num_splits), _ptr(o),
+                               _ptr(lse), _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                               _stream(stream)))
+    return o, lse
 
 
 def attn_get_device_error(stream=None):

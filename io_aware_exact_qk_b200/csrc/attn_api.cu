@@ -126,7 +126,7 @@ int record_error(int status, const char* fmt, ...) {
 const char* kernel_kind_name(int kind) {
   static const char* names[K_NUM_KINDS] = {"fwd_bf16_sm100",  "bwd_preprocess",       "bwd_bf16_sm100",
                                            "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",
-                                           "bwd_fp32_dkdv_kernel"};
+                                           "bwd_fp32_dkdv_kernel", "decode_bf16_sm100", "decode_combine"};
   return (kind >= 0 && kind < K_NUM_KINDS) ? names[kind] : "";
 }
 
@@ -162,11 +162,16 @@ LaunchScope::~LaunchScope() {
 }
 
 bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows) {
+  return encode_tma_3d_box(tmap_out, base, d, heads, rows, box_inner, 1, box_rows);
+}
+
+bool encode_tma_3d_box(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_heads,
+                       int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)box_rows};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapSwizzle swz = box_inner * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : box_inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -217,6 +222,110 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t*
   return from_cuda(launch_fwd_fp32(pb, static_cast<const float*>(q), static_cast<const float*>(k),
                                    static_cast<const float*>(v), static_cast<float*>(o), lse, s),
                    "attn_fwd (fp32 check mode) launch");
+}
+
+}  // extern "C"
+
+namespace {
+// Validation of the decoding call's shape arguments; fills `pb`.
+attn_status check_decode(const int32_t* cu_q, const int32_t* cu_k, int32_t batch, int32_t seqlen_q,
+                         int32_t seqlen_k, int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q,
+                         int32_t total_k, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                         int32_t num_splits, DecodeProblem* pb) {
+  if (d != 32 && d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {32, 64, 128}", d);
+  if (hq <= 0 || hkv <= 0) return fail(ATTN_ERR_INVALID_ARG, "head counts must be positive (hq=%d hkv=%d)", hq, hkv);
+  if (hq % hkv != 0) return fail(ATTN_ERR_UNSUPPORTED, "hq=%d is not a multiple of hkv=%d", hq, hkv);
+  if (hkv > 65535 || batch > 65535) return fail(ATTN_ERR_UNSUPPORTED, "hkv and batch must be <= 65535");
+  if (batch < 0 || total_q < 0 || total_k < 0 || num_splits < 0)
+    return fail(ATTN_ERR_INVALID_ARG, "negative batch / total_q / total_k / num_splits");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if ((cu_q == nullptr) != (cu_k == nullptr))
+    return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must both be given or both be NULL");
+  if (cu_q == nullptr) {
+    if (seqlen_q < 0 || seqlen_k < 0) return fail(ATTN_ERR_INVALID_ARG, "negative seqlen_q / seqlen_k");
+    if ((int64_t)batch * seqlen_q != total_q || (int64_t)batch * seqlen_k != total_k)
+      return fail(ATTN_ERR_INVALID_ARG, "batch mode needs total_q == batch * seqlen_q and total_k == batch * seqlen_k");
+    max_seqlen_q = seqlen_q;
+    max_seqlen_k = seqlen_k;
+  } else {
+    if ((reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u))
+      return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k are not 4-byte aligned");
+    if (max_seqlen_q < 0 || max_seqlen_k < 0 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+      return fail(ATTN_ERR_INVALID_ARG, "max_seqlen_q / max_seqlen_k out of range");
+  }
+  // one KV head's query rows (its hq/hkv heads x the newest max_seqlen_q tokens) share one
+  // 128-row tile
+  if ((int64_t)(hq / hkv) * max_seqlen_q > 128)
+    return fail(ATTN_ERR_UNSUPPORTED, "(hq / hkv) * max_seqlen_q = %lld exceeds 128 query rows per KV head",
+                (long long)(hq / hkv) * max_seqlen_q);
+  if ((int64_t)total_q * hq > (int64_t)INT32_MAX || (int64_t)total_k * hkv > (int64_t)INT32_MAX * 4)
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+  pb->cu_q = cu_q;
+  pb->cu_k = cu_k;
+  pb->batch = batch;
+  pb->seqlen_q = cu_q ? 0 : seqlen_q;
+  pb->seqlen_k = cu_q ? 0 : seqlen_k;
+  pb->max_seqlen_q = max_seqlen_q;
+  pb->max_seqlen_k = max_seqlen_k;
+  pb->total_q = total_q;
+  pb->total_k = total_k;
+  pb->hq = hq;
+  pb->hkv = hkv;
+  pb->d = d;
+  pb->scale = scale;
+  pb->causal = causal;
+  pb->num_splits = num_splits;
+  pb->varlen = cu_q != nullptr;
+  return ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd_decode(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int32_t batch, int32_t seqlen_q, int32_t seqlen_k,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q, int32_t total_k,
+                            int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal, int32_t num_splits,
+                            void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeProblem pb;
+  attn_status st = check_decode(cu_seqlens_q, cu_seqlens_k, batch, seqlen_q, seqlen_k, max_seqlen_q, max_seqlen_k,
+                                total_q, total_k, hq, hkv, d, scale, causal, num_splits, &pb);
+  if (st != ATTN_OK) return st;
+  if (total_q == 0 || batch == 0) return ok();
+  if ((st = check_ptr(q, "q")) || (st = check_ptr(o, "o")) || (st = check_ptr(lse, "lse"))) return st;
+  if (total_k > 0 && ((st = check_ptr(k, "k")) || (st = check_ptr(v, "v")))) return st;
+  const DecodeSplit sp = decode_split(pb);
+  if (sp.workspace_bytes > 0) {
+    if (workspace_bytes < sp.workspace_bytes)
+      return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes,
+                  sp.workspace_bytes);
+    if ((st = check_ptr(workspace, "workspace"))) return st;
+  }
+  // An empty key tensor still needs valid TMA descriptors: point them at q (never read).
+  const void* kk = total_k > 0 ? k : q;
+  const void* vv = total_k > 0 ? v : q;
+  if (total_k == 0) pb.total_k = 1;
+  return from_cuda(launch_decode_bf16(pb, q, kk, vv, o, lse, workspace, static_cast<cudaStream_t>(stream)),
+                   "decode launch");
+}
+
+size_t attn_fwd_decode_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q,
+                                      int32_t total_k, int32_t hq, int32_t hkv, int32_t d, int32_t varlen,
+                                      int32_t num_splits) {
+  if (batch <= 0 || total_q <= 0 || hq <= 0 || hkv <= 0 || d <= 0) return 0;
+  DecodeProblem pb{};
+  pb.batch = batch;
+  pb.max_seqlen_q = max_seqlen_q;
+  pb.max_seqlen_k = max_seqlen_k;
+  pb.total_q = total_q;
+  pb.total_k = total_k;
+  pb.hq = hq;
+  pb.hkv = hkv;
+  pb.d = d;
+  pb.varlen = varlen != 0;
+  pb.num_splits = num_splits;
+  return decode_split(pb).workspace_bytes;
 }
 
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,

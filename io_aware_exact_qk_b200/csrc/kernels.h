@@ -29,6 +29,26 @@ cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, con
                             const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                             cudaStream_t stream);
 
+// Decoding-shaped forward (split-KV): sequence b has Lq query rows (the newest positions)
+// and Lk keys.  q [Tq,hq,d], k/v [Tk,hkv,d], o [Tq,hq,d] bf16, lse [hq,Tq] f32.
+struct DecodeProblem {
+  const int32_t* cu_q;   // device prefix sums [batch + 1], or nullptr (fixed seqlen_q)
+  const int32_t* cu_k;   // device prefix sums [batch + 1], or nullptr (fixed seqlen_k)
+  int32_t batch, seqlen_q, seqlen_k, max_seqlen_q, max_seqlen_k, total_q, total_k;
+  int32_t hq, hkv, d;
+  float scale;
+  int32_t causal;
+  int32_t num_splits;    // requested key splits, 0 = chosen from the shape and the SM count
+  int32_t varlen;        // lengths come from cu_q / cu_k (only their bounds are known on the host)
+};
+struct DecodeSplit {
+  int tiles_per_split, n_splits;
+  size_t o_part_bytes, workspace_bytes;
+};
+DecodeSplit decode_split(const DecodeProblem& pb);
+cudaError_t launch_decode_bf16(const DecodeProblem& pb, const void* q, const void* k, const void* v, void* o,
+                               float* lse, void* workspace, cudaStream_t stream);
+
 // fp32 check mode (SIMT fp32 arithmetic).
 cudaError_t launch_fwd_fp32(const Problem& pb, const float* q, const float* k, const float* v, float* o,
                             float* lse, cudaStream_t stream);
@@ -47,6 +67,8 @@ enum KernelKind : int {
   K_FWD_FP32,
   K_BWD_FP32_DQ,
   K_BWD_FP32_DKDV,
+  K_DECODE_BF16,
+  K_DECODE_COMBINE,
   K_NUM_KINDS
 };
 const char* kernel_kind_name(int kind);
@@ -66,6 +88,10 @@ int record_error(int status, const char* fmt, ...);
 // [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that
 // matches a box_inner * 2-byte row (128 B or 64 B).
 bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows);
+// The same with a box spanning `box_heads` consecutive heads (box_inner x box_heads x
+// box_rows); the tile lands in shared memory as rows (token, head), head fastest.
+bool encode_tma_3d_box(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_heads,
+                       int box_rows);
 // The same over an fp32 [rows, heads, d] tensor; a 32-float (128-byte) box row uses the
 // 128-byte swizzle, any other width is unswizzled.  Used for bulk reductions.
 bool encode_tma_3d_f32(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows);

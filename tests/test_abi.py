@@ -86,3 +86,48 @@ def test_workspace_sizes(lib):
     assert lib.attn_fwd_workspace_size(4, 2048, 8192, 16, 16, 128, 0) == 0
     assert lib.attn_bwd_workspace_size(1, 0, 0, 4, 4, 64, 0) == 0
     assert lib.attn_bwd_workspace_size(2, 10, 20, 4, 2, 32, 1) == 4 * 20 * 4   # fp32 mode: D only
+
+
+def _dec(lib, **kw):
+    a = dict(q=16, k=16, v=16, cu_q=None, cu_k=None, batch=2, seqlen_q=1, seqlen_k=300, max_q=0, max_k=0,
+             total_q=2, total_k=600, hq=8, hkv=2, d=128, scale=0.088, causal=0, splits=1, o=16, lse=16, ws=None,
+             wsb=0, stream=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return lib.attn_fwd_decode(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["cu_q"]), vp(a["cu_k"]), a["batch"],
+                               a["seqlen_q"], a["seqlen_k"], a["max_q"], a["max_k"], a["total_q"], a["total_k"],
+                               a["hq"], a["hkv"], a["d"], a["scale"], a["causal"], a["splits"], vp(a["o"]),
+                               vp(a["lse"]), vp(a["ws"]), a["wsb"], vp(a["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(hq=3, hkv=2), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(hq=64, hkv=1, seqlen_q=3, total_q=6), attn.ATTN_ERR_UNSUPPORTED),   # 64 heads x 3 rows > 128
+    (dict(total_q=3), attn.ATTN_ERR_INVALID_ARG),
+    (dict(total_k=599), attn.ATTN_ERR_INVALID_ARG),
+    (dict(cu_q=0x1000), attn.ATTN_ERR_INVALID_ARG),                             # cu_k missing
+    (dict(scale=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(causal=3), attn.ATTN_ERR_INVALID_ARG),
+    (dict(splits=-1), attn.ATTN_ERR_INVALID_ARG),
+    (dict(q=None), attn.ATTN_ERR_INVALID_ARG),
+    (dict(k=0x1004), attn.ATTN_ERR_INVALID_ARG),
+    (dict(splits=3, ws=None, wsb=0), attn.ATTN_ERR_INVALID_ARG),                # needs a workspace
+])
+def test_decode_rejects_bad_arguments_on_host(lib, kw, status):
+    assert _dec(lib, **kw) == status
+    assert lib.attn_last_error_message() != b""
+
+
+def test_decode_empty_problem_is_a_no_op(lib):
+    assert _dec(lib, batch=0, total_q=0, total_k=0, q=None, k=None, v=None, o=None, lse=None) == attn.ATTN_OK
+
+
+def test_decode_workspace_sizes(lib):
+    # 1 sequence, 1 query row, 1024 keys = 8 key tiles in 4 splits of 2: partial O (fp32,
+    # 256-byte aligned) + partial LSE
+    assert lib.attn_fwd_decode_workspace_size(1, 1, 1024, 1, 1024, 8, 8, 128, 0, 4) == 4 * 8 * 128 * 4 + 4 * 8 * 4
+    assert lib.attn_fwd_decode_workspace_size(1, 1, 1024, 1, 1024, 8, 8, 128, 0, 1) == 0
+    # more splits than key tiles are clamped: 300 keys = 3 tiles
+    assert lib.attn_fwd_decode_workspace_size(2, 1, 300, 2, 600, 8, 2, 64, 1, 16) == \
+        ((3 * 2 * 8 * 64 * 4 + 255) // 256) * 256 + 3 * 8 * 2 * 4
