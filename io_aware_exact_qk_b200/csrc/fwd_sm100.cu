@@ -79,7 +79,13 @@ struct FwdCfg {
   static constexpr int B_OFINAL = B_PFULL + 2;       // 2
   static constexpr int B_OFREE = B_OFINAL + 2;       // 2
   static constexpr int NBARS = B_OFREE + 2;
-  static constexpr int DATA_BYTES = (2 + 2 * STAGES) * TILE_BYTES;
+  // Epilogue staging: each softmax warp turns its 32 O rows into coalesced stores through a
+  // 32-row slice of STG_ROWB bytes per row (half a row per pass at d = 128).
+  static constexpr int STG_ROWB = D * 2 < 128 ? D * 2 : 128;
+  static constexpr int STG_PASSES = D * 2 / STG_ROWB;
+  static constexpr int STG_WARP_BYTES = 32 * STG_ROWB;
+  static constexpr int O_STG = (2 + 2 * STAGES) * TILE_BYTES;
+  static constexpr int DATA_BYTES = O_STG + 8 * STG_WARP_BYTES;
   static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 16;
 };
 
@@ -450,21 +456,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool row_ok = qi < it.len;
-      __nv_bfloat16* orow = p.o + ((size_t)(it.seq_start + qi) * p.hq + it.h) * D;
+      // O / l as bf16, written through this warp's staging slice so that each store
+      // instruction covers whole 128-byte row segments (a thread-per-row store would touch
+      // 32 different lines per instruction).  16-byte chunk ch of staged row r sits at
+      // chunk ch ^ (r % CH), which keeps both the row-wise writes and the segment-wise reads
+      // free of bank conflicts.
+      constexpr int CH = C::STG_ROWB / 16;          // 16-byte chunks per staged row
+      constexpr int RPI = 32 / CH;                  // rows per coalesced store instruction
+      uint8_t* stg = smem + C::O_STG + warp * C::STG_WARP_BYTES;
+      const int row0 = it.q0 + t * kRows + lane_base;   // query index of the warp's first row
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-        uint32_t w[16];
+      for (int pass = 0; pass < C::STG_PASSES; ++pass) {
+        constexpr int COLS = C::STG_ROWB / 2;       // bf16 columns per pass
+        uint32_t w[COLS / 2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int c = 0; c < COLS / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + pass * COLS + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            w[c * 16 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
         }
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch)
+          *reinterpret_cast<uint4*>(stg + lane * C::STG_ROWB + ((ch ^ (lane % CH)) << 4)) =
+              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int r = i * RPI + lane / CH;
+          const int ch = lane % CH;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + r * C::STG_ROWB + ((ch ^ (r % CH)) << 4));
+          if (row0 + r < it.len)
+            *reinterpret_cast<uint4*>(p.o + ((size_t)(it.seq_start + row0 + r) * p.hq + it.h) * D + pass * COLS +
+                                      ch * 8) = v;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
