@@ -162,6 +162,21 @@ size_t attn_fwd_decode_workspace_size(int32_t batch, int32_t max_seqlen_q, int32
                                       int32_t total_q, int32_t total_k, int32_t hq, int32_t hkv,
                                       int32_t d, int32_t varlen, int32_t num_splits);
 
+/* Merge of partial results over disjoint key sets, the building block of ring attention
+ * ("相关工作" page, paper 7: each device attends its queries to the K/V block it holds,
+ * and the blocks travel around a ring).  For one row, partials (O_a, LSE_a) and
+ * (O_b, LSE_b) over disjoint keys combine exactly as the tutorial's section 修正公式
+ * combines blocks:  LSE = ln(e^LSE_a + e^LSE_b),  O = e^(LSE_a - LSE) O_a + e^(LSE_b - LSE) O_b.
+ * attn_merge_partial folds a bf16 partial (o_part [T,hq,d], lse_part [hq,T], e.g. one
+ * attn_fwd result) into the float32 accumulators o_acc [T,hq,d] and lse_acc [hq,T];
+ * first = 1 starts them from that partial (their contents are ignored).  A partial row
+ * with LSE = -inf (no visible key) contributes nothing.  attn_merge_finish writes
+ * o = bf16(o_acc) [T,hq,d].  d in {32, 64, 128}; device pointers, 16-byte aligned. */
+attn_status attn_merge_partial(float *o_acc, float *lse_acc, const void *o_part, const float *lse_part,
+                               int32_t total_tokens, int32_t hq, int32_t d, int32_t first, void *stream);
+attn_status attn_merge_finish(const float *o_acc, void *o, int32_t total_tokens, int32_t hq, int32_t d,
+                              void *stream);
+
 /* Workspace bytes attn_fwd / attn_bwd need for these shape arguments (0 = none). */
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,
                                int32_t hq, int32_t hkv, int32_t d, int32_t dtype);

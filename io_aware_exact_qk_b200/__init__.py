@@ -75,6 +75,10 @@ def load_library():
     lib.attn_fwd_decode.restype = ctypes.c_int
     lib.attn_fwd_decode_workspace_size.argtypes = [i32] * 10
     lib.attn_fwd_decode_workspace_size.restype = sz
+    lib.attn_merge_partial.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.attn_merge_partial.restype = ctypes.c_int
+    lib.attn_merge_finish.argtypes = [vp, vp, i32, i32, i32, vp]
+    lib.attn_merge_finish.restype = ctypes.c_int
     lib.attn_launch_count.argtypes = []
     lib.attn_launch_count.restype = ctypes.c_int64
     _lib = lib
@@ -234,6 +238,23 @@ def attn_fwd_decode(q, k, v, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=
                                _ptr(lse), _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                _stream(stream)))
     return o, lse
+
+
+def attn_merge_partial(o_acc, lse_acc, o_part, lse_part, first=False, stream=None):
+    """Folds a bf16 partial (o_part [T,Hq,d], lse_part [Hq,T]) over a disjoint key set into
+    the float32 accumulators o_acc [T,Hq,d], lse_acc [Hq,T] (first=True: start from it)."""
+    T, hq, d = o_part.shape
+    _check(load_library().attn_merge_partial(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), T, hq, d,
+                                             int(bool(first)), _stream(stream)))
+
+
+def attn_merge_finish(o_acc, o=None, stream=None):
+    """bf16 copy of the accumulated O."""
+    T, hq, d = o_acc.shape
+    if o is None:
+        o = torch.empty(o_acc.shape, dtype=torch.bfloat16, device=o_acc.device)
+    _check(load_library().attn_merge_finish(_ptr(o_acc), _ptr(o), T, hq, d, _stream(stream)))
+    return o
 
 
 def attn_get_device_error(stream=None):

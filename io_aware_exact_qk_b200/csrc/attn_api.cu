@@ -126,7 +126,8 @@ int record_error(int status, const char* fmt, ...) {
 const char* kernel_kind_name(int kind) {
   static const char* names[K_NUM_KINDS] = {"fwd_bf16_sm100",  "bwd_preprocess",       "bwd_bf16_sm100",
                                            "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",
-                                           "bwd_fp32_dkdv_kernel", "decode_bf16_sm100", "decode_combine"};
+                                           "bwd_fp32_dkdv_kernel", "decode_bf16_sm100", "decode_combine",
+                                           "merge_partial",   "merge_finish"};
   return (kind >= 0 && kind < K_NUM_KINDS) ? names[kind] : "";
 }
 
@@ -308,6 +309,34 @@ attn_status attn_fwd_decode(const void* q, const void* k, const void* v, const i
   if (total_k == 0) pb.total_k = 1;
   return from_cuda(launch_decode_bf16(pb, q, kk, vv, o, lse, workspace, static_cast<cudaStream_t>(stream)),
                    "decode launch");
+}
+
+attn_status attn_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                               int32_t total_tokens, int32_t hq, int32_t d, int32_t first, void* stream) {
+  if (d != 32 && d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {32, 64, 128}", d);
+  if (total_tokens < 0 || hq <= 0) return fail(ATTN_ERR_INVALID_ARG, "need total_tokens >= 0 and hq > 0");
+  if (first != 0 && first != 1) return fail(ATTN_ERR_INVALID_ARG, "first must be 0 or 1");
+  if ((int64_t)total_tokens * hq > (int64_t)INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  if (total_tokens == 0) return ok();
+  attn_status st;
+  if ((st = check_ptr(o_acc, "o_acc")) || (st = check_ptr(lse_acc, "lse_acc")) || (st = check_ptr(o_part, "o_part")) ||
+      (st = check_ptr(lse_part, "lse_part")))
+    return st;
+  return from_cuda(launch_merge_partial(o_acc, lse_acc, o_part, lse_part, total_tokens, hq, d, first,
+                                        static_cast<cudaStream_t>(stream)),
+                   "merge launch");
+}
+
+attn_status attn_merge_finish(const float* o_acc, void* o, int32_t total_tokens, int32_t hq, int32_t d,
+                              void* stream) {
+  if (d != 32 && d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {32, 64, 128}", d);
+  if (total_tokens < 0 || hq <= 0) return fail(ATTN_ERR_INVALID_ARG, "need total_tokens >= 0 and hq > 0");
+  if ((int64_t)total_tokens * hq > (int64_t)INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  if (total_tokens == 0) return ok();
+  attn_status st;
+  if ((st = check_ptr(o_acc, "o_acc")) || (st = check_ptr(o, "o"))) return st;
+  return from_cuda(launch_merge_finish(o_acc, o, total_tokens, hq, d, static_cast<cudaStream_t>(stream)),
+                   "merge launch");
 }
 
 size_t attn_fwd_decode_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q,

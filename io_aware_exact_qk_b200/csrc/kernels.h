@@ -49,6 +49,12 @@ DecodeSplit decode_split(const DecodeProblem& pb);
 cudaError_t launch_decode_bf16(const DecodeProblem& pb, const void* q, const void* k, const void* v, void* o,
                                float* lse, void* workspace, cudaStream_t stream);
 
+// Merge of partial results over disjoint key sets (ring attention): o_acc [T,hq,d] f32,
+// lse_acc [hq,T] f32 accumulate bf16 partials o_part [T,hq,d] / lse_part [hq,T].
+cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                                 int total_tokens, int hq, int d, int first, cudaStream_t stream);
+cudaError_t launch_merge_finish(const float* o_acc, void* o, int total_tokens, int hq, int d, cudaStream_t stream);
+
 // fp32 check mode (SIMT fp32 arithmetic).
 cudaError_t launch_fwd_fp32(const Problem& pb, const float* q, const float* k, const float* v, float* o,
                             float* lse, cudaStream_t stream);
@@ -69,6 +75,8 @@ enum KernelKind : int {
   K_BWD_FP32_DKDV,
   K_DECODE_BF16,
   K_DECODE_COMBINE,
+  K_MERGE_PARTIAL,
+  K_MERGE_FINISH,
   K_NUM_KINDS
 };
 const char* kernel_kind_name(int kind);

@@ -1,0 +1,105 @@
+"""Ring attention's GPU arithmetic: the forward on chunk pairs and the merge kernels.
+
+This run has one GPU, so the ranks of the ring are emulated in turn in one process: for
+every rank the hops of ``ring_schedule`` are executed with the library's kernels
+(attn_fwd on the (query chunk, K/V chunk) pair, attn_merge_partial, attn_merge_finish),
+and the rows of all ranks together must match the fp64 oracle over the whole sequences
+with the forward's tolerances.  The point-to-point passing of the blocks between real
+ranks is covered by the gloo test on the CPU; the driver itself runs here as a one-rank
+NCCL group.
+"""
+import datetime
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import attn_workloads as W
+import io_aware_exact_qk_b200 as attn
+import oracle
+from io_aware_exact_qk_b200.ring import ring_attn_fwd, ring_schedule
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(batch, N, hq, hkv, d, seed):
+    w = W.custom("ring", [N] * batch, hq, hkv, d, False, seed)
+    q, k, v, _, cu = W.make_inputs(w, with_grad=False)
+    return w, q, k, v, cu
+
+
+def _chunks(t, batch, N, world):
+    n = N // world
+    t = t.reshape(batch, N, *t.shape[1:])
+    return [t[:, r * n:(r + 1) * n].reshape(batch * n, *t.shape[2:]).contiguous().cuda() for r in range(world)]
+
+
+@pytest.mark.parametrize("world,causal,d", [(2, False, 128), (4, True, 128), (3, True, 64), (5, False, 32)])
+def test_emulated_ring_matches_full_attention(world, causal, d):
+    batch, n, hq, hkv = 2, 256 if d == 128 else 200, 8, 2
+    N = world * n
+    w, q, k, v, cu = _inputs(batch, N, hq, hkv, d, 3100 + world)
+    qs, ks, vs = (_chunks(t, batch, N, world) for t in (q, k, v))
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, cu.numpy(), scale=w.scale, causal=causal)
+    o_ref = o_ref.reshape(batch, N, hq, d)
+    lse_ref = lse_ref.reshape(hq, batch, N)
+    for r in range(world):
+        o_acc = torch.empty(batch * n, hq, d, dtype=torch.float32, device="cuda")
+        lse_acc = torch.empty(hq, batch * n, dtype=torch.float32, device="cuda")
+        first = True
+        for j, kind in ring_schedule(r, world, causal):
+            if kind is None:
+                continue
+            o_p, lse_p = attn.attn_fwd(qs[r], ks[j], vs[j], scale=w.scale, causal=kind == "causal", batch=batch)
+            attn.attn_merge_partial(o_acc, lse_acc, o_p, lse_p, first=first)
+            first = False
+        o = attn.attn_merge_finish(o_acc)
+        attn.attn_get_device_error()
+        mine = slice(r * n, (r + 1) * n)
+        parity.check_fwd_bf16(parity.to_np(o).reshape(batch, n, hq, d), parity.to_np(lse_acc).reshape(hq, batch, n),
+                              o_ref[:, mine], lse_ref[:, :, mine], tag=f"rank {r}")
+
+
+def test_merge_kernel_edge_cases():
+    T, hq, d = 37, 4, 128
+    g = torch.Generator().manual_seed(5)
+    o_acc = torch.randn(T, hq, d, generator=g).cuda()
+    lse_acc = torch.randn(hq, T, generator=g).cuda()
+    o_p = torch.randn(T, hq, d, generator=g).to(torch.bfloat16).cuda()
+    # a partial without visible keys leaves the accumulator as it is
+    before = (o_acc.clone(), lse_acc.clone())
+    attn.attn_merge_partial(o_acc, lse_acc, o_p, torch.full((hq, T), -np.inf, device="cuda"))
+    torch.testing.assert_close(o_acc, before[0], rtol=0, atol=0)
+    torch.testing.assert_close(lse_acc, before[1], rtol=0, atol=0)
+    # first=True starts from the partial; equal LSEs average the two partials
+    lse_p = torch.randn(hq, T, generator=g).cuda()
+    attn.attn_merge_partial(o_acc, lse_acc, o_p, lse_p, first=True)
+    torch.testing.assert_close(o_acc, o_p.float(), rtol=0, atol=0)
+    torch.testing.assert_close(lse_acc, lse_p, rtol=0, atol=0)
+    o_q = torch.randn(T, hq, d, generator=g).to(torch.bfloat16).cuda()
+    attn.attn_merge_partial(o_acc, lse_acc, o_q, lse_p)
+    torch.testing.assert_close(o_acc, (o_p.float() + o_q.float()) / 2, rtol=1e-6, atol=1e-6)
+    torch.testing.assert_close(lse_acc, lse_p + float(np.log(2.0)), rtol=1e-6, atol=1e-6)
+    assert torch.equal(attn.attn_merge_finish(o_acc), o_acc.to(torch.bfloat16))
+    attn.attn_get_device_error()
+
+
+def test_driver_as_a_one_rank_nccl_group():
+    """The driver's own code path (defaults = the library's kernels) on one rank."""
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        batch, N, hq, hkv, d = 2, 384, 8, 4, 128
+        w, q, k, v, cu = _inputs(batch, N, hq, hkv, d, 3200)
+        o, lse = ring_attn_fwd(q.cuda(), k.cuda(), v.cuda(), batch, scale=w.scale, causal=True)
+        attn.attn_get_device_error()
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, cu.numpy(), scale=w.scale, causal=True)
+        parity.check_fwd_bf16(o, lse, o_ref, lse_ref, tag="one-rank ring")
+    finally:
+        dist.destroy_process_group()

@@ -1,0 +1,113 @@
+"""The ring-attention driver over a real multi-process group (gloo on CPU).
+
+Each rank holds one chunk of every sequence and runs ``ring_attn_fwd``, the same driver
+the GPUs run, with its two compute steps swapped for CPU stand-ins (the local attention
+from the fp64 oracle, the merge in float64 numpy) -- the schedule, the masks of every hop
+and the point-to-point passing of the K/V blocks are what is under test here.  The rows
+gathered from all ranks must equal the oracle's forward over the whole sequences.
+"""
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from io_aware_exact_qk_b200.ring import ring_schedule
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _local_oracle(batch, scale):
+    def f(q, k, v, causal):
+        n = q.shape[0] // batch
+        cu = np.arange(batch + 1, dtype=np.int32) * n
+        o, lse = oracle.attn_fwd(q.numpy(), k.numpy(), v.numpy(), cu, scale=scale, causal=causal, threads=1)
+        return torch.from_numpy(o), torch.from_numpy(lse)
+    return f
+
+
+def _merge64(o_acc, lse_acc, o_p, lse_p, first):
+    o_p, lse_p = o_p.double(), lse_p.double()
+    if first:
+        o_acc.copy_(o_p)
+        lse_acc.copy_(lse_p)
+        return
+    la, lp = lse_acc.clone(), lse_p
+    m = torch.maximum(la, lp)
+    wa = torch.where(la == -np.inf, 0.0, torch.exp(la - m))
+    wp = torch.where(lp == -np.inf, 0.0, torch.exp(lp - m))
+    s = wa + wp
+    # [hq, T] weights -> [T, hq, 1]
+    o_acc.mul_((wa / s).T[:, :, None]).add_(o_p * (wp / s).T[:, :, None])
+    lse_acc.copy_(m + torch.log(s))
+
+
+def _worker(rank, world, port, batch, n, hq, hkv, d, causal, out):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        from io_aware_exact_qk_b200.ring import ring_attn_fwd
+        g = torch.Generator().manual_seed(77)
+        N = world * n
+        q = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
+        k = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+        v = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+        mine = slice(rank * n, (rank + 1) * n)
+        qc, kc, vc = (t[:, mine].reshape(batch * n, t.shape[2], d).contiguous() for t in (q, k, v))
+        scale = 1.0 / np.sqrt(d)
+        o, lse = ring_attn_fwd(qc, kc, vc, batch, scale=scale, causal=causal, local_fwd=_local_oracle(batch, scale),
+                               merge=_merge64, finish=lambda oa: oa, acc_dtype=torch.float64)
+        out[rank] = (o.numpy(), lse.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_forward_equals_full_attention(world, causal):
+    batch, n, hq, hkv, d = 2, 5, 4, 2, 8
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as man:
+        out = man.dict()
+        procs = [ctx.Process(target=_worker, args=(r, world, port, batch, n, hq, hkv, d, causal, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    g = torch.Generator().manual_seed(77)
+    N = world * n
+    q = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
+    k = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+    v = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+    cu = np.arange(batch + 1, dtype=np.int32) * N
+    o_ref, lse_ref = oracle.attn_fwd(q.reshape(-1, hq, d).numpy(), k.reshape(-1, hkv, d).numpy(),
+                                     v.reshape(-1, hkv, d).numpy(), cu, causal=causal)
+    o_ref = o_ref.reshape(batch, N, hq, d)
+    lse_ref = lse_ref.reshape(hq, batch, N)
+    for r in range(world):
+        o, lse = res[r]
+        mine = slice(r * n, (r + 1) * n)
+        np.testing.assert_allclose(o.reshape(batch, n, hq, d), o_ref[:, mine], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse.reshape(hq, batch, n), lse_ref[:, :, mine], rtol=0, atol=1e-12)
+
+
+def test_ring_schedule_visits_every_block_once():
+    for world in (1, 2, 5):
+        for causal in (False, True):
+            for r in range(world):
+                hops = ring_schedule(r, world, causal)
+                assert sorted(j for j, _ in hops) == list(range(world))
+                assert hops[0] == (r, "causal" if causal else "full")   # own block first
+                for j, kind in hops:
+                    assert kind == ("full" if not causal or j < r else ("causal" if j == r else None))
