@@ -189,6 +189,14 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank contributes its own device-timed milliseconds."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------------------
 # GPU side
 # ---------------------------------------------------------------------------------------
@@ -265,10 +273,7 @@ def run_ours(args, rank, world, local_rank):
     per_kernel = attn.attn_profile_collect()
     attn.attn_get_device_error()
     total_ms = sum(s.elapsed_time(e) for s, e in events)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
 
     # ---- end to end: host buffers, copies inside the timed region ----
@@ -298,10 +303,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     attn.attn_get_device_error()
     e2e_ms = e2e_start.elapsed_time(e2e_end)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * flops_step * args.steps / (float(t.item()) / 1e3) / 1e12
+    e2e_value = world * flops_step * args.steps / (max_over_ranks(e2e_ms, world, dev) / 1e3) / 1e12
 
     if rank != 0:
         return
@@ -446,10 +448,7 @@ def run_decode(args, rank, world, local_rank):
     per_kernel = attn.attn_profile_collect()
     attn.attn_get_device_error()
     total_ms = sum(s_.elapsed_time(e_) for s_, e_ in events)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     value = world * w.hbm_bytes() * args.steps / (total_ms / 1e3) / 1e9
     if args.quick:
         if rank == 0:
@@ -474,10 +473,7 @@ def run_decode(args, rank, world, local_rank):
     e1.record(stream)
     barrier()
     attn.attn_get_device_error()
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * w.hbm_bytes() * args.steps / (float(t.item()) / 1e3) / 1e9
+    e2e_value = world * w.hbm_bytes() * args.steps / (max_over_ranks(e0.elapsed_time(e1), world, dev) / 1e3) / 1e9
     if rank != 0:
         return
     peaks = load_peaks()
