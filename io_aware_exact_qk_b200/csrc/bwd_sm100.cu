@@ -521,25 +521,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue: warps 0-3 write dV, warps 4-7 write dK = scale * acc ------
     if (ok && mbar_wait(bar(C::B_DONE), 0, abort_flag)) {
       tc_fence_after();
-      const bool row_ok = kj < len;
-      const size_t orow = ((size_t)(seq_start + kj) * p.hkv + g) * D;
-      __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + orow;
+      // Every MMA has completed, so the Q/dO ring is idle: each warp stages its 32 rows
+      // there (half a row per pass at d = 128) and stores whole 128-byte row segments per
+      // instruction instead of 32 scattered 16-byte pieces.  Chunk ch of staged row r sits
+      // at ch ^ (r % CH): conflict-free row writes and segment reads.
+      constexpr int ROWB = D * 2 < 128 ? D * 2 : 128;
+      constexpr int COLS = ROWB / 2;               // bf16 columns per pass
+      constexpr int CH = ROWB / 16;                // 16-byte chunks per staged row
+      constexpr int RPI = 32 / CH;                 // rows per coalesced store instruction
+      static_assert(8 * 32 * ROWB <= 2 * C::STAGES * C::Q_TILE_BYTES, "staging fits in the Q/dO ring");
+      uint8_t* stg = smem + C::O_Q + warp * 32 * ROWB;
+      __nv_bfloat16* base = half == 0 ? p.dv : p.dk;
       const float mul = half == 0 ? 1.f : p.scale;
       const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
+      const int key0 = kv0 + lane_base;            // key index of the warp's first row
 #pragma unroll
-      for (int cb = 0; cb < D; cb += 32) {
-        uint32_t r[32];
-        tmem_ld32(trow + col + cb, r);
-        tmem_wait_ld();
-        if (row_ok) {
-          uint32_t w[16];
+      for (int pass = 0; pass < D * 2 / ROWB; ++pass) {
+        uint32_t w[COLS / 2];
+#pragma unroll
+        for (int c = 0; c < COLS / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(trow + col + pass * COLS + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
-          uint4* o4 = reinterpret_cast<uint4*>(dst + cb);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            w[c * 16 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
         }
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch)
+          *reinterpret_cast<uint4*>(stg + lane * ROWB + ((ch ^ (lane % CH)) << 4)) =
+              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int r = i * RPI + lane / CH;
+          const int ch = lane % CH;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + r * ROWB + ((ch ^ (r % CH)) << 4));
+          if (key0 + r < len)
+            *reinterpret_cast<uint4*>(base + ((size_t)(seq_start + key0 + r) * p.hkv + g) * D + pass * COLS + ch * 8) = v;
+        }
+        __syncwarp();
       }
     }
   } else if (warp < 12) {
