@@ -12,12 +12,14 @@
 // Three launches on the caller's stream:
 //   1. bwd_preprocess   D = rowsum(dO o O) into the workspace and zero the fp32 dQ
 //                       accumulator (HBM-bound).
-//   2. bwd_main         one CTA per (128-key tile, kv head, sequence).  The CTA keeps
-//                       K_j, V_j in shared memory and dK_j, dV_j in TMEM, and walks the
-//                       query tiles of every query head of its GQA group (so dK/dV need
-//                       no atomics).  Per query tile i (BM rows):
+//   2. bwd_main         persistent, one CTA per SM; a work item is a (128-key tile, kv
+//                       head, sequence), claimed from a global counter in a fixed order.
+//                       For its item the CTA keeps K_j in shared memory (two buffers: the
+//                       next item's K_j loads while this one runs), V_j and dK_j, dV_j in
+//                       TMEM, and walks the query tiles of every query head of the GQA
+//                       group (so dK/dV need no atomics).  Per query tile i (BM rows):
 //                         S^T  = K_j Q_i^T            (tcgen05, TMEM fp32)
-//                         dP^T = V_j dO_i^T           (tcgen05, TMEM fp32)
+//                         dP^T = V_j dO_i^T           (tcgen05, A = V_j from TMEM)
 //                         P^T, dS^T on the compute warpgroup, one key row per thread,
 //                           written back as bf16 over S^T / dP^T, dS^T also to SMEM
 //                         dV  += P^T dO_i             (A from TMEM)
@@ -41,8 +43,11 @@
 // dQ_i = dS K_j (M = 128 query rows, N = d): 128 + 128 + 4 d <= 512 columns.
 //
 // Warp roles (448 threads): two compute warpgroups, each owning half of the query columns
-// of every step (P^T, dS^T) and one of the dK / dV epilogues; a dQ drain warpgroup; a TMA
-// producer warp (+ LSE / D rows into SMEM, one step ahead); an MMA issuer warp.
+// of every step (P^T, dS^T) and one of the dK / dV epilogues (which also load the next
+// item's V_j into TMEM); a dQ drain warpgroup; a TMA producer warp that claims the items
+// (+ LSE / D rows into SMEM, one step ahead); an MMA issuer warp.  Across items the
+// pipelines keep running: the next item's K_j and first Q / dO tiles load during the
+// current item, and its first products start while the epilogue drains dK / dV.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -51,14 +56,18 @@ namespace attn {
 namespace {
 
 constexpr int kKeys = 128;   // keys per CTA == TMEM lanes
+constexpr int kItemSlots = 4;  // ring of work-item indices the producer hands to the other roles
 constexpr int kThreads = 448;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct BwdCfg {
   static constexpr bool DQT = (D == 128);          // dQ^T form (see file comment)
-  static constexpr bool VT = DQT;                 // V_j held in TMEM, dP^T as a TS product
-  static constexpr int STAGES = DQT ? (VT ? 4 : 3) : 2;   // Q_i / dO_i / LSE_i / D_i ring depth
+  static constexpr bool VT = true;                // V_j held in TMEM, dP^T as a TS product
+  static constexpr int STAGES = DQT ? 3 : 2;      // Q_i / dO_i / LSE_i / D_i ring depth
+  // K_j (and V_j when it is not in TMEM) buffers: two, so the next work item's tile loads
+  // while the current one runs.
+  static constexpr int KV_BUFS = 2;
   static constexpr int BM = DQT ? 64 : 128;       // query rows per step
   static constexpr int HALF = BM / 2;             // query columns per compute warpgroup
   static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span of Q/K/V/dO rows (bytes)
@@ -73,26 +82,28 @@ struct BwdCfg {
   static constexpr int Q_TILE_BYTES = BM * D * 2;
   static constexpr int DS_PANEL_BYTES = kKeys * 128;  // dS^T: 128 key rows x 64 queries (bf16)
   static constexpr int DS_BYTES = kKeys * BM * 2;
-  // TMEM columns.  d = 128: two dP^T buffers, so dP^T(n+1) can be issued before dK(n)
-  // reads dS^T(n) out of the other one, and a single dQ^T slot (its drain copies it out
-  // at once):  S^T [0,64) dP^T[0] [64,128) dP^T[1] [128,192) dV [192,320) dK [320,448)
-  // dQ^T [448,512).  d <= 64: one dP^T buffer and two dQ slots:
-  //   S^T [0,BM) dP^T [BM,2BM) dV, dK (d each) then two dQ slots of d columns.
+  // TMEM columns.  V_j (bf16 pairs, D/2 columns) is the A operand of dP^T; one dP^T
+  // buffer.  d = 128:  V [0,64) S^T [64,128) dP^T [128,192) dV [192,320) dK [320,448)
+  // dQ^T [448,512).  d = 64:  S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384)
+  // dQ [384,448) V [448,480).  d = 32: S^T, dP^T as for d = 64, dV [256,288) dK [288,320),
+  // two dQ slots [320,384), V [384,400).
   static constexpr int NDPT = (DQT && !VT) ? 2 : 1;  // dP^T buffers
-  static constexpr int NDQ = DQT ? 1 : 2;            // dQ slots
-  static constexpr int T_V = 0;                      // V_j as a bf16 A operand: D/2 columns
-  static constexpr int V_COLS = VT ? D / 2 : 0;
-  static constexpr int T_ST = V_COLS;
+  static constexpr int NDQ = (DQT || D == 64) ? 1 : 2;   // dQ slots (d = 64: room for V)
+  static constexpr int V_COLS = VT ? D / 2 : 0;      // V_j as a bf16 A operand: D/2 columns
+  // d = 128 puts V first; d <= 64 after the accumulators (every accumulator 64-aligned)
+  static constexpr int T_ST = DQT ? V_COLS : 0;
   static constexpr int T_DPT = T_ST + BM;            // dP^T buffer b at T_DPT + b * BM
   static constexpr int T_DV = T_DPT + NDPT * BM;
   static constexpr int T_DK = T_DV + D;
   static constexpr int T_DQ = T_DK + D;              // NDQ slots of DQ_COLS
   static constexpr int DQ_COLS = DQT ? BM : D;
-  static_assert(T_DQ + NDQ * DQ_COLS <= 512, "TMEM budget");
+  static constexpr int T_V = DQT ? 0 : T_DQ + NDQ * DQ_COLS;
+  static_assert(T_DQ + NDQ * DQ_COLS + (DQT ? 0 : V_COLS) <= 512, "TMEM budget");
   // shared memory map (offsets from the 1024-aligned base)
-  static constexpr int O_K = 0;
-  static constexpr int O_V = O_K + KV_TILE_BYTES;
-  static constexpr int O_Q = O_V + (VT ? 0 : KV_TILE_BYTES);   // STAGES
+  static constexpr int KVB_BYTES = (VT ? 1 : 2) * KV_TILE_BYTES;   // one K (+ V) buffer
+  static constexpr int O_K = 0;                                 // buffer b at O_K + b * KVB_BYTES
+  static constexpr int O_V = O_K + KV_TILE_BYTES;               // inside a buffer
+  static constexpr int O_Q = O_K + KV_BUFS * KVB_BYTES;         // STAGES
   static constexpr int O_DO = O_Q + STAGES * Q_TILE_BYTES;      // STAGES
   static constexpr int O_DS = O_DO + STAGES * Q_TILE_BYTES;     // 2 buffers
   // LSE_i * log2 e and D_i rows live in LSLOTS slots (slot n % LSLOTS for step n), each
@@ -111,8 +122,9 @@ struct BwdCfg {
   static constexpr int STG_BYTES = STG_ROWS * D * 4;
   static constexpr int O_BAR = O_STG + STG_BYTES;
   // barriers
-  static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;                  // STAGES
+  static constexpr int B_KFULL = 0;                  // KV_BUFS (2 reserved)
+  static constexpr int B_KEMPTY = 2;                 // KV_BUFS (2 reserved)
+  static constexpr int B_QFULL = 4;                  // STAGES
   static constexpr int B_QEMPTY = B_QFULL + STAGES;  // STAGES
   static constexpr int B_LFULL = B_QEMPTY + STAGES;  // LSLOTS
   static constexpr int B_ST = B_LFULL + LSLOTS;
@@ -124,8 +136,19 @@ struct BwdCfg {
   static constexpr int B_DQEMPTY = B_DQFULL + 2;     // 2
   static constexpr int B_DONE = B_DQEMPTY + 2;
   static constexpr int B_VT = B_DONE + 1;            // V_j written into TMEM
-  static constexpr int NBARS = B_VT + 1;
-  static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 16;
+  static constexpr int B_EPI = B_VT + 1;             // dK, dV read out of TMEM
+  static constexpr int B_IFULL = B_EPI + 1;          // kItemSlots: item index written
+  static constexpr int B_IEMPTY = B_IFULL + kItemSlots;   // kItemSlots: read by every role
+  static constexpr int NBARS = B_IEMPTY + kItemSlots;
+  // after the barriers: TMEM address, abort flag, the item-index ring
+  static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 8 + 4 * kItemSlots;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // the dK / dV epilogue stages 32 rows per compute warp in the finished item's K buffer:
+  // row segments of up to 128 bytes, as much as the buffer holds
+  static constexpr int EPI_ROWB_CAP = KVB_BYTES / (8 * 32);
+  static constexpr int EPI_ROWB = (D * 2 < 128 ? D * 2 : 128) < EPI_ROWB_CAP ? (D * 2 < 128 ? D * 2 : 128)
+                                                                             : EPI_ROWB_CAP;
+  static_assert(EPI_ROWB >= 32 && 8 * 32 * EPI_ROWB <= KVB_BYTES, "epilogue staging fits in a K buffer");
 };
 
 struct BwdParams {
@@ -137,6 +160,9 @@ struct BwdParams {
   const float* lse;      // [hq, T]
   const float* dd;       // [hq, T]
   const __nv_bfloat16* v;   // [T, hkv, d] (read directly when V_j lives in TMEM)
+  int32_t batch, n_kt, n_items;   // work items: (key tile, kv head, sequence)
+  int32_t heads_per_group;         // causal order: heads whose Q / dO stream fits in L2
+  int* item_counter;               // next unclaimed item (zeroed by the preprocess kernel)
   float* dq_acc;         // [T, hq, d]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -150,6 +176,51 @@ struct StepIter {
     *i = i_begin + n % steps_per_head;
   }
 };
+
+// One work item: a 128-key tile of one kv head of one sequence.
+struct BItem {
+  int g, seq_start, len, kv0, n_steps;   // n_steps == 0: nothing to do
+  StepIter it;
+};
+
+// Work item number idx.  The CTAs are persistent (one per SM) and claim items in this
+// order from a global counter, so each takes the next one as soon as it is free.  With
+// heads_per_group > 0 (causal, d = 128) the order is heaviest-first (key tile 0 is seen
+// by every query) within groups of heads whose Q / dO stream fits in about 32 MB of L2,
+// so that the items in flight share what they read and lighter items fill in at the end;
+// otherwise the key tiles of one head are consecutive.
+template <int BM>
+__device__ __forceinline__ BItem bitem_from(const BwdParams& p, int idx) {
+  BItem w;
+  w.n_steps = 0;
+  w.g = w.seq_start = w.len = w.kv0 = 0;
+  w.it.G = w.it.i_begin = w.it.n_q = w.it.steps_per_head = 0;
+  if (idx < 0 || idx >= p.n_items) return w;
+  int jt, r;
+  if (p.causal && p.heads_per_group > 0) {
+    const int pairs = p.hkv * p.batch;
+    const int per_grp = p.n_kt * p.heads_per_group;
+    const int grp = idx / per_grp, rem = idx % per_grp;
+    const int ng = min(p.heads_per_group, pairs - grp * p.heads_per_group);
+    jt = rem / ng;
+    r = grp * p.heads_per_group + rem % ng;
+  } else {
+    jt = idx % p.n_kt;
+    r = idx / p.n_kt;
+  }
+  w.g = r % p.hkv;
+  const int b = r / p.hkv;
+  w.seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
+  w.len = p.cu_seqlens ? p.cu_seqlens[b + 1] - w.seq_start : p.seqlen;
+  w.kv0 = jt * kKeys;
+  if (w.kv0 >= w.len) return w;
+  w.it.G = p.hq / p.hkv;
+  w.it.n_q = (w.len + BM - 1) / BM;
+  w.it.i_begin = p.causal ? w.kv0 / BM : 0;
+  w.it.steps_per_head = w.it.n_q - w.it.i_begin;
+  w.n_steps = w.it.G * w.it.steps_per_head;
+  return w;
+}
 
 // Byte offset of the 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled panel.
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
@@ -179,30 +250,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::O_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_items = reinterpret_cast<volatile int*>(tmem_slot + 2);
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int jt = blockIdx.x;       // key tile: the tiles of one head run together (L2 reuse)
-  const int g = blockIdx.y;        // kv head
-  const int b = blockIdx.z;        // sequence
-  const int seq_start = p.cu_seqlens ? p.cu_seqlens[b] : b * p.seqlen;
-  const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - seq_start : p.seqlen;
-  const int kv0 = jt * kKeys;
-  if (kv0 >= len) return;
-  StepIter it;
-  it.G = p.hq / p.hkv;
-  it.n_q = (len + BM - 1) / BM;
-  it.i_begin = p.causal ? kv0 / BM : 0;
-  it.steps_per_head = it.n_q - it.i_begin;
-  const int n_steps = it.G * it.steps_per_head;
+  // The producer claims items and hands their indices to the other roles through the
+  // s_items ring; every role walks the same items in the same order.  Per-step barriers
+  // count steps over all the CTA's items; per-item ones (K buffers, V in TMEM, done,
+  // epilogue) count non-empty items.  next_item(k) returns the k-th claimed index (or
+  // -1 after a failed wait); an index >= n_items ends the walk.
+  auto next_item = [&](int k) -> int {
+    const int slot = k % kItemSlots;
+    if (!mbar_wait(bar(C::B_IFULL + slot), (k / kItemSlots) & 1, abort_flag)) return -1;
+    const int idx = s_items[slot];
+    __syncwarp(__activemask());
+    if ((threadIdx.x & 31) == __ffs(__activemask()) - 1) mbar_arrive(bar(C::B_IEMPTY + slot));
+    return idx;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
-      // warp-level arrivals: one per compute warp (PT, DS) or drain warp (DQEMPTY)
-      if (i == C::B_PT || i == C::B_DS) cnt = 8;
+      // warp-level arrivals: one per compute warp (PT, DS, K buffer free, epilogue read
+      // out) or drain warp (DQEMPTY), one per first-warpgroup warp for V in TMEM
+      if (i == C::B_PT || i == C::B_DS || i == C::B_EPI || i == C::B_KEMPTY || i == C::B_KEMPTY + 1) cnt = 8;
       if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1 || i == C::B_VT) cnt = 4;
+      // item slots are read by the MMA warp, the 8 compute warps and the 4 drain warps
+      if (i >= C::B_IEMPTY && i < C::B_IEMPTY + kItemSlots) cnt = 13;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -225,59 +300,85 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 12) {
-    // ---------------- producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per step ----------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::B_KV), (C::VT ? 1 : 2) * C::KV_TILE_BYTES);
-      for (int pn = 0; pn < C::NPANEL; ++pn) {
-        tma_load_3d(sbase + C::O_K + pn * C::KV_PANEL_BYTES, &tmK, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
-        if (!C::VT)
-          tma_load_3d(sbase + C::O_V + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KV), pn * C::PANEL, g, seq_start + kv0);
-      }
-    }
+    // ---------------- producer: K_j (V_j) per item; Q_i, dO_i, LSE_i, D_i per step ---------
     // LSE_i * log2(e) and D_i of the next step are loaded into registers one step ahead,
     // so their global-memory latency overlaps the wait for a free stage.  Query rows past
     // the sequence get LSE = +inf (P = 0 there without a mask) and D = 0.
     constexpr int PER_LANE = BM / 32;
     float nl[PER_LANE], nd[PER_LANE];
-    auto fetch = [&](int n) {
-      int h, i;
-      it.head_tile(n, g, &h, &i);
-#pragma unroll
-      for (int e = 0; e < PER_LANE; ++e) {
-        const int qi = i * BM + e * 32 + lane;
-        const bool ok = qi < len;
-        const size_t idx = (size_t)h * p.total_tokens + seq_start + (ok ? qi : 0);
-        nl[e] = ok ? p.lse[idx] * kLog2e : INFINITY;
-        nd[e] = ok ? p.dd[idx] : 0.f;
-      }
-    };
-    fetch(0);
-    for (int n = 0; n < n_steps; ++n) {
-      const int s = n % C::STAGES;
-      const int ls = n % C::LSLOTS;
-      // Stage s is free once dK(n - STAGES) is done; LSE slot ls was last read by step
-      // n - LSLOTS, whose dS finished before dK(n - LSLOTS), so it is free too.
-      if (!mbar_wait(bar(C::B_QEMPTY + s), ((n / C::STAGES) & 1) ^ 1, abort_flag)) break;
-      int h, i;
-      it.head_tile(n, g, &h, &i);
-      const int q0 = i * BM;
-#pragma unroll
-      for (int e = 0; e < PER_LANE; ++e) {
-        s_lse[ls * BM + e * 32 + lane] = nl[e];
-        s_dd[ls * BM + e * 32 + lane] = nd[e];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_LFULL + ls));
-      if (n + 1 < n_steps) fetch(n + 1);
+    int ng = 0;          // steps so far (all items)
+    int in = 0;          // non-empty items so far
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      // claim the next item and hand its index to the other roles
+      const int slot = k % kItemSlots;
+      if (!mbar_wait(bar(C::B_IEMPTY + slot), ((k / kItemSlots) & 1) ^ 1, abort_flag)) break;
+      int idx = 0;
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
+        idx = atomicAdd(p.item_counter, 1);
+        s_items[slot] = idx;
+      }
+      idx = __shfl_sync(0xffffffffu, idx, 0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_IFULL + slot));
+      if (idx >= p.n_items) break;
+      const BItem w = bitem_from<BM>(p, idx);
+      if (w.n_steps == 0) continue;
+      const int kb = in % C::KV_BUFS;
+      // The buffer is free once the item that used it last has finished its epilogue.
+      if (!mbar_wait(bar(C::B_KEMPTY + kb), ((in / C::KV_BUFS) & 1) ^ 1, abort_flag)) break;
+      if (lane == 0) {
+        const uint32_t kbase = sbase + C::O_K + kb * C::KVB_BYTES;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + kb), C::KVB_BYTES);
         for (int pn = 0; pn < C::NPANEL; ++pn) {
-          tma_load_3d(sbase + C::O_Q + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmQ, bar(C::B_QFULL + s),
-                      pn * C::PANEL, h, seq_start + q0);
-          tma_load_3d(sbase + C::O_DO + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmDO, bar(C::B_QFULL + s),
-                      pn * C::PANEL, h, seq_start + q0);
+          tma_load_3d(kbase + pn * C::KV_PANEL_BYTES, &tmK, bar(C::B_KFULL + kb), pn * C::PANEL, w.g,
+                      w.seq_start + w.kv0);
+          if (!C::VT)
+            tma_load_3d(kbase + (C::O_V - C::O_K) + pn * C::KV_PANEL_BYTES, &tmV, bar(C::B_KFULL + kb),
+                        pn * C::PANEL, w.g, w.seq_start + w.kv0);
         }
       }
+      auto fetch = [&](int n) {
+        int h, i;
+        w.it.head_tile(n, w.g, &h, &i);
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) {
+          const int qi = i * BM + e * 32 + lane;
+          const bool in_seq = qi < w.len;
+          const size_t idx = (size_t)h * p.total_tokens + w.seq_start + (in_seq ? qi : 0);
+          nl[e] = in_seq ? p.lse[idx] * kLog2e : INFINITY;
+          nd[e] = in_seq ? p.dd[idx] : 0.f;
+        }
+      };
+      fetch(0);
+      for (int n = 0; n < w.n_steps; ++n, ++ng) {
+        const int s = ng % C::STAGES;
+        const int ls = ng % C::LSLOTS;
+        // Stage s is free once dK(ng - STAGES) is done; LSE slot ls was last read by step
+        // ng - LSLOTS, whose dS finished before dK(ng - LSLOTS), so it is free too.
+        if (!mbar_wait(bar(C::B_QEMPTY + s), ((ng / C::STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        int h, i;
+        w.it.head_tile(n, w.g, &h, &i);
+        const int q0 = i * BM;
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) {
+          s_lse[ls * BM + e * 32 + lane] = nl[e];
+          s_dd[ls * BM + e * 32 + lane] = nd[e];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_LFULL + ls));
+        if (n + 1 < w.n_steps) fetch(n + 1);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+            tma_load_3d(sbase + C::O_Q + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmQ, bar(C::B_QFULL + s),
+                        pn * C::PANEL, h, w.seq_start + q0);
+            tma_load_3d(sbase + C::O_DO + s * C::Q_TILE_BYTES + pn * C::Q_PANEL_BYTES, &tmDO, bar(C::B_QFULL + s),
+                        pn * C::PANEL, h, w.seq_start + q0);
+          }
+        }
+      }
+      ++in;
     }
   } else if (warp == 13) {
     // ---------------- MMA issuer ----------------
@@ -292,9 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Every operand descriptor is a base descriptor (computed once, or once per ring
       // stage) advanced by a compile-time offset, so issuing one MMA takes a few
       // instructions; the issue rate of this single thread bounds the tensor core here.
-      const uint64_t k_kmaj = smem_desc(sbase + C::O_K, 16, C::SBO, C::SWZ);               // K, K-major
-      const uint64_t v_kmaj = smem_desc(sbase + C::O_V, 16, C::SBO, C::SWZ);               // V, K-major
-      const uint64_t k_mn = smem_desc(sbase + C::O_K, C::KV_PANEL_BYTES, C::SBO, C::SWZ);  // K^T operand
+      // K / V descriptors of buffer 0; buffer kb adds kb * KVB_BYTES
+      const uint64_t k_kmaj0 = smem_desc(sbase + C::O_K, 16, C::SBO, C::SWZ);               // K, K-major
+      const uint64_t v_kmaj0 = smem_desc(sbase + C::O_V, 16, C::SBO, C::SWZ);               // V, K-major
+      const uint64_t k_mn0 = smem_desc(sbase + C::O_K, C::KV_PANEL_BYTES, C::SBO, C::SWZ);  // K^T operand
+      uint64_t k_kmaj = k_kmaj0, v_kmaj = v_kmaj0, k_mn = k_mn0;
       const uint64_t q_kmaj = smem_desc(sbase + C::O_Q, 16, C::SBO, C::SWZ);
       const uint64_t do_kmaj = smem_desc(sbase + C::O_DO, 16, C::SBO, C::SWZ);
       const uint64_t q_mn = smem_desc(sbase + C::O_Q, C::Q_PANEL_BYTES, C::SBO, C::SWZ);
@@ -344,108 +447,153 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss(tmem + d_col, sd, kd, id_dq, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag) && mbar_wait(bar(C::B_QFULL), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(k_kmaj, q_kmaj, C::T_ST);
-        mma_commit(bar(C::B_ST));
-        ok = !C::VT || mbar_wait(bar(C::B_VT), 0, abort_flag);
-      }
-      if (ok) {
-        tc_fence_after();
-        issue_dpt(do_kmaj, C::T_DPT);
-        mma_commit(bar(C::B_DPT));
-      }
-      // Order per step n (dP^T buffer db = n & 1 when NDPT == 2, else 0):
-      //   [PT(n)] dV(n); S^T(n+1); NDPT == 2: dP^T(n+1) into the other buffer;
-      //   [DS(n)] dK(n) (reads dS^T(n) from buffer db); [dQ slot free] dQ(n);
-      //   NDPT == 1: dP^T(n+1) here, once dK(n) has been issued.
-      for (int n = 0; ok && n < n_steps; ++n) {
-        const int s = n % C::STAGES;
-        const int s1 = (n + 1) % C::STAGES;
-        const int b2 = n & 1;
-        const int db = C::NDPT == 2 ? b2 : 0;
-        const int db1 = C::NDPT == 2 ? (b2 ^ 1) : 0;
-        const int qslot = C::NDQ == 2 ? b2 : 0;
-        const uint32_t qpar = C::NDQ == 2 ? (((n >> 1) & 1) ^ 1) : (uint32_t)((n & 1) ^ 1);
-        const bool more = n + 1 < n_steps;
-        if (!mbar_wait(bar(C::B_PT), n & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_grad(C::T_ST, stage(do_mn, s), C::T_DV, n > 0);                 // dV += P^T dO
-        if (more) {
-          if (!mbar_wait(bar(C::B_QFULL + s1), ((n + 1) / C::STAGES) & 1, abort_flag)) break;
+      int ng0 = 0;         // steps before the current item (all items)
+      int in = 0;          // non-empty items so far
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = next_item(k);
+        if (idx < 0 || idx >= p.n_items) break;
+        const BItem w = bitem_from<BM>(p, idx);
+        if (w.n_steps == 0) continue;
+        const int kb = in % C::KV_BUFS;
+        k_kmaj = desc_advance(k_kmaj0, (uint32_t)kb * C::KVB_BYTES);
+        v_kmaj = desc_advance(v_kmaj0, (uint32_t)kb * C::KVB_BYTES);
+        k_mn = desc_advance(k_mn0, (uint32_t)kb * C::KVB_BYTES);
+        const int s0 = ng0 % C::STAGES;
+        ok = mbar_wait(bar(C::B_KFULL + kb), (in / C::KV_BUFS) & 1, abort_flag) &&
+             mbar_wait(bar(C::B_QFULL + s0), (ng0 / C::STAGES) & 1, abort_flag);
+        if (ok) {
           tc_fence_after();
-          issue_sdp(k_kmaj, stage(q_kmaj, s1), C::T_ST);                      // S^T for the next step
+          issue_sdp(k_kmaj, stage(q_kmaj, s0), C::T_ST);
           mma_commit(bar(C::B_ST));
-          if (C::NDPT == 2) {
-            issue_dpt(stage(do_kmaj, s1), C::T_DPT + db1 * BM);               // dP^T(n+1)
-            mma_commit(bar(C::B_DPT + db1));
+          // V_j of this item in TMEM (its compute warps load it after the previous item)
+          ok = !C::VT || mbar_wait(bar(C::B_VT), in & 1, abort_flag);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_dpt(stage(do_kmaj, s0), C::T_DPT + (C::NDPT == 2 ? (ng0 & 1) * BM : 0));
+          mma_commit(bar(C::B_DPT + (C::NDPT == 2 ? (ng0 & 1) : 0)));
+        }
+        // Order per step n (global step ng; dP^T buffer db = ng & 1 when NDPT == 2, else 0):
+        //   [PT(ng)] dV(ng); S^T(ng+1); NDPT == 2: dP^T(ng+1) into the other buffer;
+        //   [DS(ng)] dK(ng) (reads dS^T(ng) from buffer db); [dQ slot free] dQ(ng);
+        //   NDPT == 1: dP^T(ng+1) here, once dK(ng) has been issued.
+        // The first dV / dK of an item overwrite the accumulators, so they wait until the
+        // previous item's epilogue has read them out.
+        for (int n = 0; ok && n < w.n_steps; ++n) {
+          const int ng = ng0 + n;
+          const int s = ng % C::STAGES;
+          const int s1 = (ng + 1) % C::STAGES;
+          const int b2 = ng & 1;
+          const int db = C::NDPT == 2 ? b2 : 0;
+          const int db1 = C::NDPT == 2 ? (b2 ^ 1) : 0;
+          const int qslot = C::NDQ == 2 ? b2 : 0;
+          const uint32_t qpar = C::NDQ == 2 ? (((ng >> 1) & 1) ^ 1) : (uint32_t)((ng & 1) ^ 1);
+          const bool more = n + 1 < w.n_steps;
+          if (!mbar_wait(bar(C::B_PT), ng & 1, abort_flag)) { ok = false; break; }
+          if (n == 0 && in > 0 && !mbar_wait(bar(C::B_EPI), (in - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_grad(C::T_ST, stage(do_mn, s), C::T_DV, n > 0);                 // dV += P^T dO
+          if (more) {
+            if (!mbar_wait(bar(C::B_QFULL + s1), ((ng + 1) / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_sdp(k_kmaj, stage(q_kmaj, s1), C::T_ST);                      // S^T for the next step
+            mma_commit(bar(C::B_ST));
+            if (C::NDPT == 2) {
+              issue_dpt(stage(do_kmaj, s1), C::T_DPT + db1 * BM);               // dP^T(ng+1)
+              mma_commit(bar(C::B_DPT + db1));
+            }
+          }
+          if (!mbar_wait(bar(C::B_DS), ng & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_grad(C::T_DPT + db * BM, stage(q_mn, s), C::T_DK, n > 0);       // dK += dS^T Q
+          mma_commit(bar(C::B_QEMPTY + s));
+          if (!mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                           // dQ_i partial
+          mma_commit(bar(C::B_DQFULL + qslot));
+          mma_commit(bar(C::B_DSFREE + b2));
+          if (C::NDPT == 1 && more) {
+            issue_dpt(stage(do_kmaj, s1), C::T_DPT);                            // dP^T for the next step
+            mma_commit(bar(C::B_DPT));
           }
         }
-        if (!mbar_wait(bar(C::B_DS), n & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_grad(C::T_DPT + db * BM, stage(q_mn, s), C::T_DK, n > 0);       // dK += dS^T Q
-        mma_commit(bar(C::B_QEMPTY + s));
-        if (!mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) break;
-        tc_fence_after();
-        issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                           // dQ_i partial
-        mma_commit(bar(C::B_DQFULL + qslot));
-        mma_commit(bar(C::B_DSFREE + b2));
-        if (C::NDPT == 1 && more) {
-          issue_dpt(stage(do_kmaj, s1), C::T_DPT);                            // dP^T for the next step
-          mma_commit(bar(C::B_DPT));
-        }
+        mma_commit(bar(C::B_DONE));    // every product of this item (dK, dV final)
+        ng0 += w.n_steps;
+        ++in;
       }
-      mma_commit(bar(C::B_DONE));
     }
   } else if (warp < 8) {
     // ---------------- compute: P^T, dS^T for one key row and half of the query columns ----
     const int half = warp >> 2;                   // 0: columns [0, HALF), 1: [HALF, BM)
     const int lane_base = (warp & 3) * 32;
     const int kr = lane_base + lane;              // key row inside the tile
-    const int kj = kv0 + kr;                      // key index inside the sequence
     const int c0 = half * HALF;                   // first query column of this thread
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     const float sl2 = p.scale_log2;
+    int ng0 = 0;         // steps before the current item (all items)
+    int in = 0;          // non-empty items so far
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+    const int idx = next_item(k);
+    if (idx < 0 || idx >= p.n_items) break;
+    const BItem w = bitem_from<BM>(p, idx);
+    if (w.n_steps == 0) continue;
+    const int g = w.g, seq_start = w.seq_start, len = w.len, kv0 = w.kv0;
+    const int kj = kv0 + kr;                      // key index inside the sequence
     if (C::VT && half == 0) {
       // V_j row kr, bf16 pairs as they lie in memory (element 2c in the low half of column
-      // c), is the A operand of dP^T; rows past the sequence are zero.
+      // c), is the A operand of dP^T; rows past the sequence are zero.  (The previous
+      // item's products are all done: its epilogue waited for them.)
       const uint4* vrow = reinterpret_cast<const uint4*>(p.v + ((size_t)(seq_start + kj) * p.hkv + g) * D);
+      if constexpr (C::V_COLS >= 32) {
 #pragma unroll
-      for (int cb = 0; cb < C::V_COLS; cb += 32) {
-        uint32_t w[32];
+        for (int cb = 0; cb < C::V_COLS; cb += 32) {
+          uint32_t w[32];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 x = kj < len ? vrow[cb / 4 + e] : make_uint4(0u, 0u, 0u, 0u);
+          for (int e = 0; e < 8; ++e) {
+            const uint4 x = kj < len ? vrow[cb / 4 + e] : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * e] = x.x;
+            w[4 * e + 1] = x.y;
+            w[4 * e + 2] = x.z;
+            w[4 * e + 3] = x.w;
+          }
+          tmem_st32(trow + C::T_V + cb, w);
+        }
+      } else {   // d = 32: a 64-byte row, 16 columns
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint4 x = kj < len ? vrow[e] : make_uint4(0u, 0u, 0u, 0u);
           w[4 * e] = x.x;
           w[4 * e + 1] = x.y;
           w[4 * e + 2] = x.z;
           w[4 * e + 3] = x.w;
         }
-        tmem_st32(trow + C::T_V + cb, w);
+        tmem_st16(trow + C::T_V, w);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_VT));
     }
-    bool ok = true;
-    for (int n = 0; n < n_steps; ++n) {
-      const int ls = n % C::LSLOTS;
-      const int b2 = n & 1;
+    for (int n = 0; n < w.n_steps; ++n) {
+      const int ng = ng0 + n;
+      const int ls = ng % C::LSLOTS;
+      const int b2 = ng & 1;
       const int db = C::NDPT == 2 ? b2 : 0;                           // dP^T buffer
-      const uint32_t dpar = C::NDPT == 2 ? ((n >> 1) & 1) : (uint32_t)(n & 1);
+      const uint32_t dpar = C::NDPT == 2 ? ((ng >> 1) & 1) : (uint32_t)(ng & 1);
       const uint32_t t_dpt = C::T_DPT + db * BM;
       int h, i;
-      it.head_tile(n, g, &h, &i);
+      w.it.head_tile(n, g, &h, &i);
       const int q0 = i * BM;
       // Columns c < c_lo are hidden by the causal mask; a key past the sequence hides all.
       // (Query rows past the sequence carry LSE = +inf, so they come out as P = 0.)
       int c_lo = p.causal ? kj - q0 : 0;
       if (kj >= len) c_lo = BM;
       const bool masked = c_lo > c0;
-      if (!mbar_wait(bar(C::B_LFULL + ls), (n / C::LSLOTS) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(C::B_ST), n & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_LFULL + ls), (ng / C::LSLOTS) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_ST), ng & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const float4* lse4 = reinterpret_cast<const float4*>(s_lse + ls * BM + c0);
       const float4* dd4 = reinterpret_cast<const float4*>(s_dd + ls * BM + c0);
@@ -483,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_PT));
       // dS^T = P^T o (dP^T - D): to TMEM (over dP^T) and to the swizzled SMEM buffer
-      if (!mbar_wait(bar(C::B_DSFREE + b2), ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(C::B_DSFREE + b2), ((ng >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       if (!mbar_wait(bar(C::B_DPT + db), dpar, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint8_t* ds_smem = smem + C::O_DS + b2 * C::DS_BYTES;
@@ -519,18 +667,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(C::B_DS));
     }
     // ---------------- epilogue: warps 0-3 write dV, warps 4-7 write dK = scale * acc ------
-    if (ok && mbar_wait(bar(C::B_DONE), 0, abort_flag)) {
+    if (!ok || !mbar_wait(bar(C::B_DONE), in & 1, abort_flag)) { ok = false; break; }
+    {
       tc_fence_after();
-      // Every MMA has completed, so the Q/dO ring is idle: each warp stages its 32 rows
-      // there (half a row per pass at d = 128) and stores whole 128-byte row segments per
-      // instruction instead of 32 scattered 16-byte pieces.  Chunk ch of staged row r sits
-      // at ch ^ (r % CH): conflict-free row writes and segment reads.
-      constexpr int ROWB = D * 2 < 128 ? D * 2 : 128;
+      // Every product of the item has completed, so its K buffer is idle: each warp stages
+      // its 32 rows there (half a row per pass at d = 128) and stores whole 128-byte row
+      // segments per instruction instead of 32 scattered 16-byte pieces.  Chunk ch of
+      // staged row r sits at ch ^ (r % CH): conflict-free row writes and segment reads.
+      constexpr int ROWB = C::EPI_ROWB;
       constexpr int COLS = ROWB / 2;               // bf16 columns per pass
       constexpr int CH = ROWB / 16;                // 16-byte chunks per staged row
       constexpr int RPI = 32 / CH;                 // rows per coalesced store instruction
-      static_assert(8 * 32 * ROWB <= 2 * C::STAGES * C::Q_TILE_BYTES, "staging fits in the Q/dO ring");
-      uint8_t* stg = smem + C::O_Q + warp * 32 * ROWB;
+      const int kb = in % C::KV_BUFS;
+      uint8_t* stg = smem + C::O_K + kb * C::KVB_BYTES + warp * 32 * ROWB;
       __nv_bfloat16* base = half == 0 ? p.dv : p.dk;
       const float mul = half == 0 ? 1.f : p.scale;
       const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
@@ -538,14 +687,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int pass = 0; pass < D * 2 / ROWB; ++pass) {
         uint32_t w[COLS / 2];
+        if constexpr (COLS >= 32) {
 #pragma unroll
-        for (int c = 0; c < COLS / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(trow + col + pass * COLS + c * 32, r);
+          for (int c = 0; c < COLS / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(trow + col + pass * COLS + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[c * 16 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+          }
+        } else {   // 16 columns per pass
+          uint32_t r[16];
+          tmem_ld16(trow + col + pass * COLS, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[c * 16 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+          for (int e = 0; e < 8; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
         }
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch)
@@ -562,18 +720,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
+      // dK / dV have been read out of TMEM: the next item's first products may overwrite
+      // them.  The K buffer is free for the producer once these generic accesses are
+      // ordered before its next (async-proxy) write.
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(C::B_EPI));
+        mbar_arrive(bar(C::B_KEMPTY + kb));
+      }
+    }
+    ng0 += w.n_steps;
+    ++in;
     }
   } else if (warp < 12) {
     // ---------------- dQ drain: TMEM partial -> fp32 atomics into the accumulator ---------
     const int lane_base = (warp & 3) * 32;
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
-    for (int n = 0; n < n_steps; ++n) {
-      const int b2 = C::NDQ == 2 ? (n & 1) : 0;                    // dQ slot
-      const uint32_t par = C::NDQ == 2 ? ((n >> 1) & 1) : (uint32_t)(n & 1);
+    int ng = 0;          // steps so far (all items)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+    const int idx = next_item(k);
+    if (idx < 0 || idx >= p.n_items) break;
+    const BItem w = bitem_from<BM>(p, idx);
+    const int seq_start = w.seq_start;
+    for (int n = 0; n < w.n_steps; ++n, ++ng) {
+      const int b2 = C::NDQ == 2 ? (ng & 1) : 0;                   // dQ slot
+      const uint32_t par = C::NDQ == 2 ? ((ng >> 1) & 1) : (uint32_t)(ng & 1);
       int h, i;
-      it.head_tile(n, g, &h, &i);
+      w.it.head_tile(n, w.g, &h, &i);
       const int q0 = i * BM;
-      if (!mbar_wait(bar(C::B_DQFULL + b2), par, abort_flag)) break;
+      if (!mbar_wait(bar(C::B_DQFULL + b2), par, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t r[C::DQ_COLS / 32][32];
 #pragma unroll
@@ -632,6 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    }
   }
 
   if (warp == 8 && lane == 0) bulk_wait_group0();   // bulk reductions complete
@@ -649,8 +828,9 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout, int64_t rows, int hq,
                                                       int total_tokens, float* __restrict__ dd,
-                                                      float* __restrict__ dq_acc) {
+                                                      float* __restrict__ dq_acc, int* __restrict__ item_counter) {
   constexpr int TPR = D / 8;   // threads per row
+  if (blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;   // the main kernel's work-item counter
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
   // The loop condition is uniform over each warp (it tests the warp's first row), so the
@@ -718,8 +898,10 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   using C = BwdCfg<D>;
   const size_t T = (size_t)pb.total_tokens;
   float* dd = static_cast<float*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                           (((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255));
+  const size_t dbytes = ((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255;
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbytes);
+  int* item_counter = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + dbytes +
+                                             T * (size_t)pb.hq * (size_t)D * sizeof(float));
   const int64_t rows = (int64_t)T * pb.hq;
   {
     const int64_t threads = rows * (D / 8);
@@ -727,7 +909,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
     LaunchScope scope(K_BWD_PREPROCESS, stream);
     bwd_preprocess<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                    static_cast<const __nv_bfloat16*>(dout), rows, pb.hq,
-                                                   pb.total_tokens, dd, dq_acc);
+                                                   pb.total_tokens, dd, dq_acc, item_counter);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -751,12 +933,29 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   p.lse = lse;
   p.dd = dd;
   p.v = static_cast<const __nv_bfloat16*>(v);
+  p.batch = pb.batch;
+  p.n_kt = (pb.max_seqlen + kKeys - 1) / kKeys;
+  const int64_t items = (int64_t)p.n_kt * pb.hkv * pb.batch;
+  if (items > INT32_MAX) return cudaErrorInvalidValue;
+  p.n_items = (int)items;
+  // Causal order: heaviest-first in groups of heads whose Q and dO together stay within
+  // ~32 MB of L2.  Measured on B200 it pays at d = 128 (64-query steps: an item is twice as
+  // many steps, long enough to hide its boundary) and loses at d <= 64, where the key
+  // tiles of one head in turn are faster.
+  p.heads_per_group = -1;
+  if (pb.causal && D == 128) {
+    const int64_t head_bytes = (int64_t)(pb.hq / pb.hkv) * pb.max_seqlen * D * 2 * 2;
+    const int64_t pairs = (int64_t)pb.hkv * pb.batch;
+    p.heads_per_group = (int)std::max<int64_t>(1, std::min<int64_t>(pairs, (32ll << 20) / std::max<int64_t>(head_bytes, 1)));
+  }
+  p.item_counter = item_counter;
   p.dq_acc = dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   cudaError_t e = cudaFuncSetAttribute(bwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((pb.max_seqlen + kKeys - 1) / kKeys, pb.hkv, pb.batch);
+  // persistent: one CTA per SM (shared memory allows no more) walking its item list
+  const int grid = (int)std::min<int64_t>(items, sm_count());
   {
     LaunchScope scope(K_BWD_BF16, stream);
     bwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
@@ -776,7 +975,7 @@ size_t bwd_bf16_workspace_bytes(const Problem& pb) {
   const size_t T = (size_t)pb.total_tokens;
   const size_t dbytes = ((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255;   // D [hq, T]
   const size_t qacc = T * (size_t)pb.hq * (size_t)pb.d * sizeof(float);             // dQ accumulator
-  return dbytes + qacc;
+  return dbytes + qacc + 256;                                                       // + item counter
 }
 
 cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, const void* o,

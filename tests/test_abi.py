@@ -75,7 +75,7 @@ def test_empty_problem_is_a_no_op(lib):
 def test_bwd_rejects_small_workspace(lib):
     vp = ctypes.c_void_p
     need = lib.attn_bwd_workspace_size(1, 8, 8, 2, 2, 64, 0)
-    assert need == ((2 * 8 * 4 + 255) // 256) * 256 + 8 * 2 * 64 * 4
+    assert need == ((2 * 8 * 4 + 255) // 256) * 256 + 8 * 2 * 64 * 4 + 256   # D, dQ accumulator, item counter
     st = lib.attn_bwd(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), None, 1, 8, 8, 8, 2, 2, 64, 0.125, 0, 0,
                       vp(16), vp(16), vp(16), vp(16), need - 1, None)
     assert st == attn.ATTN_ERR_INVALID_ARG
