@@ -79,7 +79,10 @@ typedef enum {
 
 /* Forward.  Writes o [T,hq,d] and lse [hq,T].
  * Defined by: tutorial sections 标准注意力三步 (the result), 分块 / Online Softmax 技巧
- * (how it is reached) and 前向 (only O and the row statistics are stored). */
+ * (how it is reached) and 前向 (only O and the row statistics are stored).
+ * Workspace (bf16 mode): attn_fwd_workspace_size() = 256 bytes, the counter from which the
+ * persistent kernel's CTAs claim work items; it is reset on the stream before each launch,
+ * so calls that overlap (other streams) need workspaces of their own. */
 attn_status attn_fwd(const void *q, const void *k, const void *v,
                      const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
                      int32_t max_seqlen, int32_t total_tokens,

@@ -207,8 +207,6 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t*
                      int32_t seqlen, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d,
                      float scale, int32_t causal, int32_t dtype, void* o, float* lse, void* workspace,
                      size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   Problem pb;
   attn_status st = check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal,
                                 dtype, &pb);
@@ -217,9 +215,15 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t*
   if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
       (st = check_ptr(o, "o")) || (st = check_ptr(lse, "lse")))
     return st;
+  if (dtype == ATTN_BF16) {
+    if (workspace_bytes < kFwdWorkspaceBytes)
+      return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes,
+                  kFwdWorkspaceBytes);
+    if ((st = check_ptr(workspace, "workspace"))) return st;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == ATTN_BF16)
-    return from_cuda(launch_fwd_bf16(pb, q, k, v, o, lse, s), "attn_fwd launch");
+    return from_cuda(launch_fwd_bf16(pb, q, k, v, o, lse, workspace, s), "attn_fwd launch");
   return from_cuda(launch_fwd_fp32(pb, static_cast<const float*>(q), static_cast<const float*>(k),
                                    static_cast<const float*>(v), static_cast<float*>(o), lse, s),
                    "attn_fwd (fp32 check mode) launch");
@@ -359,8 +363,8 @@ size_t attn_fwd_decode_workspace_size(int32_t batch, int32_t max_seqlen_q, int32
 
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
                                int32_t d, int32_t dtype) {
-  (void)batch, (void)max_seqlen, (void)total_tokens, (void)hq, (void)hkv, (void)d, (void)dtype;
-  return 0;
+  (void)batch, (void)max_seqlen, (void)hq, (void)hkv, (void)d;
+  return (dtype == ATTN_BF16 && total_tokens > 0) ? kFwdWorkspaceBytes : 0;   // the work-item counter
 }
 
 size_t attn_bwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,

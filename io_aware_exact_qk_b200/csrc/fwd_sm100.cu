@@ -23,9 +23,10 @@
 // consistently, so the result is exact up to rounding.  (The concept page lists this
 // "conditional rescaling" among the Blackwell techniques, 已知局限.)
 //
-// Persistent schedule: one CTA per SM walks a static list of work items, heaviest first
-// under the causal mask (zig-zag over CTAs so every CTA gets a similar total), pairs of one
-// head adjacent otherwise (their K/V stream is shared through L2).  All pipelines run
+// Persistent schedule: one CTA per SM claims work items from a global counter in a fixed
+// order -- heaviest first under the causal mask, within groups of heads whose K/V fit in
+// L2; pairs of one head adjacent otherwise (their K/V stream is shared through L2).  All
+// pipelines run
 // across items: the next item's Q load and its first QK^T MMAs overlap the current item's
 // epilogue, and the K/V ring never drains.  Under the causal mask a query tile only
 // visits key tiles it can see, so the lower tile of an item skips the last key tile.
@@ -55,6 +56,7 @@ constexpr float kRescaleSkip = 8.0f;       // log2 units, see file comment
 constexpr uint32_t kEmuPairs = 0x22u;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
+constexpr int kItemSlots = 4;  // ring of work-item indices the producer hands to the other roles
 
 template <int D>
 struct FwdCfg {
@@ -78,7 +80,9 @@ struct FwdCfg {
   static constexpr int B_PFULL = B_SFULL + 2;        // 2
   static constexpr int B_OFINAL = B_PFULL + 2;       // 2
   static constexpr int B_OFREE = B_OFINAL + 2;       // 2
-  static constexpr int NBARS = B_OFREE + 2;
+  static constexpr int B_IFULL = B_OFREE + 2;        // kItemSlots: item index written
+  static constexpr int B_IEMPTY = B_IFULL + kItemSlots;   // kItemSlots: read by MMA + softmax warps
+  static constexpr int NBARS = B_IEMPTY + kItemSlots;
   // Epilogue staging: each softmax warp turns its 32 O rows into coalesced stores through a
   // 32-row slice of STG_ROWB bytes per row (half a row per pass at d = 128).
   static constexpr int STG_ROWB = D * 2 < 128 ? D * 2 : 128;
@@ -86,7 +90,9 @@ struct FwdCfg {
   static constexpr int STG_WARP_BYTES = 32 * STG_ROWB;
   static constexpr int O_STG = (2 + 2 * STAGES) * TILE_BYTES;
   static constexpr int DATA_BYTES = O_STG + 8 * STG_WARP_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 16;
+  // after the barriers: TMEM address, abort flag, the item-index ring
+  static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 8 + 4 * kItemSlots;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct FwdParams {
@@ -98,6 +104,8 @@ struct FwdParams {
   int32_t causal;
   __nv_bfloat16* o;
   float* lse;
+  int32_t heads_per_group;   // causal order: (head, sequence) pairs whose K / V fit in L2
+  int* item_counter;         // next unclaimed item (zeroed before the launch)
 };
 
 // One work item: two query tiles of one head of one sequence.
@@ -107,23 +115,29 @@ struct Item {
   int nkv;     // key tiles loaded for the item, max(n[0], n[1])
 };
 
-__device__ __forceinline__ Item make_item(const FwdParams& p, int k) {
-  // k-th item of this CTA.  Causal: heaviest first, zig-zag over CTAs.  Otherwise the
-  // pairs of one head are consecutive.
-  const int G = gridDim.x;
-  const int idx = k * G + ((p.causal && (k & 1)) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+// Work item number idx.  The CTAs are persistent (one per SM) and claim items in this
+// order from a global counter, so each takes the next one as soon as it is free.  Causal:
+// heaviest first (the last query tiles see the most keys) within groups of
+// (head, sequence) pairs whose K / V fit in about 32 MB of L2, so that the items in flight
+// share what they stream, and lighter items fill in at the end.  Otherwise the pairs of
+// one head are consecutive (their K / V stream is shared through L2).
+__device__ __forceinline__ Item item_from(const FwdParams& p, int idx) {
   Item it;
-  if (idx >= p.n_items) {   // the last round is partial
+  if (idx < 0 || idx >= p.n_items) {
     it.h = it.b = it.seq_start = it.len = it.q0 = 0;
     it.n[0] = it.n[1] = it.nkv = 0;
     return it;
   }
   int pair;
   if (p.causal) {
-    it.h = idx % p.hq;
-    const int t = idx / p.hq;
-    it.b = t % p.batch;
-    pair = p.n_pairs - 1 - t / p.batch;
+    const int pairs = p.hq * p.batch;
+    const int per_grp = p.n_pairs * p.heads_per_group;
+    const int grp = idx / per_grp, rem = idx % per_grp;
+    const int ng = min(p.heads_per_group, pairs - grp * p.heads_per_group);
+    pair = p.n_pairs - 1 - rem / ng;
+    const int r = grp * p.heads_per_group + rem % ng;
+    it.h = r % p.hq;
+    it.b = r / p.hq;
   } else {
     pair = idx % p.n_pairs;
     const int t = idx / p.n_pairs;
@@ -160,12 +174,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_items = reinterpret_cast<volatile int*>(tmem_slot + 2);
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Every CTA walks the same number of rounds; indices past the item list are empty items.
-  const int n_mine = (p.n_items + (int)gridDim.x - 1) / (int)gridDim.x;
+  // The producer claims items and hands their indices to the MMA issuer and the softmax
+  // warps through the s_items ring, so all roles walk the same items in the same order.
+  // next_item(k) returns the k-th claimed index (-1 after a failed wait); an index
+  // >= n_items ends the walk.
+  auto next_item = [&](int k) -> int {
+    const int slot = k % kItemSlots;
+    if (!mbar_wait(bar(C::B_IFULL + slot), (k / kItemSlots) & 1, abort_flag)) return -1;
+    const int idx = s_items[slot];
+    __syncwarp(__activemask());
+    if ((threadIdx.x & 31) == __ffs(__activemask()) - 1) mbar_arrive(bar(C::B_IEMPTY + slot));
+    return idx;
+  };
 
   if (threadIdx.x == 0) {
     // sequences longer than max_seqlen would not be covered by the item list
@@ -177,7 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < C::NBARS; ++i) {
       // P-ready and O-free are arrived on once per softmax warp (after __syncwarp)
       const bool per_warp = (i == C::B_PFULL || i == C::B_PFULL + 1 || i == C::B_OFREE || i == C::B_OFREE + 1);
-      mbar_init(bar(i), per_warp ? 4u : 1u);
+      // an item slot is read by the MMA issuer and the 8 softmax warps
+      const bool slot_read = i >= C::B_IEMPTY && i < C::B_IEMPTY + kItemSlots;
+      mbar_init(bar(i), slot_read ? 9u : (per_warp ? 4u : 1u));
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -201,8 +228,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv = 0, qi = 0;   // K/V tiles and non-empty items so far
       bool ok = true;
-      for (int k = 0; ok && k < n_mine; ++k) {
-        const Item it = make_item(p, k);
+      for (int k = 0; ok; ++k) {
+        // claim the next item and hand its index to the other roles
+        const int slot = k % kItemSlots;
+        if (!mbar_wait(bar(C::B_IEMPTY + slot), ((k / kItemSlots) & 1) ^ 1, abort_flag)) break;
+        const int idx = atomicAdd(p.item_counter, 1);
+        s_items[slot] = idx;
+        mbar_arrive(bar(C::B_IFULL + slot));
+        if (idx >= p.n_items) break;
+        const Item it = item_from(p, idx);
         if (it.nkv == 0) continue;
         const int hk = it.h / (p.hq / p.hkv);
         if (!mbar_wait(bar(C::B_QEMPTY), (qi & 1) ^ 1, abort_flag)) break;
@@ -263,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pc[2] = {0, 0};   // P_t tiles consumed
       uint32_t om[2] = {0, 0};   // items started per query tile (for the O-free handshake)
       bool ok = true;
-      for (int k = 0; ok && k < n_mine; ++k) {
-        const Item it = make_item(p, k);
+      for (int k = 0; ok; ++k) {
+        const int idx = next_item(k);
+        if (idx < 0 || idx >= p.n_items) break;
+        const Item it = item_from(p, idx);
         if (it.nkv == 0) continue;
         int s_left = it.n[0] + it.n[1];   // QK^T MMAs still to issue; Q is free after the last
         ok = mbar_wait(bar(C::B_QFULL), qi & 1, abort_flag);
@@ -325,8 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, oc = 0;   // S_t tiles and items consumed by this warpgroup
     bool ok = true;
-    for (int k = 0; ok && k < n_mine; ++k) {
-      const Item it = make_item(p, k);
+    for (int k = 0; ok; ++k) {
+      const int idx = next_item(k);
+      if (idx < 0 || idx >= p.n_items) break;
+      const Item it = item_from(p, idx);
       const int n_t = it.n[t];
       if (n_t == 0) continue;
       const int qi = it.q0 + t * kRows + lane_base + lane;   // query index inside the sequence
@@ -529,7 +567,7 @@ int sm_count_fwd() {
 
 template <int D>
 cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const void* v, void* o, float* lse,
-                         cudaStream_t stream) {
+                         void* workspace, cudaStream_t stream) {
   using C = FwdCfg<D>;
   alignas(64) CUtensorMap tq, tk, tv;
   if (!encode_tma_3d(&tq, q, D, pb.hq, pb.total_tokens, C::PANEL, kRows) ||
@@ -553,7 +591,14 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
   p.causal = pb.causal;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  // causal order: (head, sequence) pairs whose K and V together stay within ~32 MB of L2
+  const int64_t kv_bytes = (int64_t)pb.max_seqlen * D * 2 * 2;
+  p.heads_per_group = (int)std::max<int64_t>(
+      1, std::min<int64_t>((int64_t)pb.hq * pb.batch, (32ll << 20) / std::max<int64_t>(kv_bytes, 1)));
+  p.item_counter = static_cast<int*>(workspace);
+  cudaError_t e = cudaMemsetAsync(p.item_counter, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<int64_t>(items, sm_count_fwd());
   LaunchScope scope(K_FWD_BF16, stream);
@@ -564,12 +609,12 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, void* o, float* lse,
-                            cudaStream_t stream) {
+                            void* workspace, cudaStream_t stream) {
   if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
   switch (pb.d) {
-    case 32: return launch_fwd_d<32>(pb, q, k, v, o, lse, stream);
-    case 64: return launch_fwd_d<64>(pb, q, k, v, o, lse, stream);
-    case 128: return launch_fwd_d<128>(pb, q, k, v, o, lse, stream);
+    case 32: return launch_fwd_d<32>(pb, q, k, v, o, lse, workspace, stream);
+    case 64: return launch_fwd_d<64>(pb, q, k, v, o, lse, workspace, stream);
+    case 128: return launch_fwd_d<128>(pb, q, k, v, o, lse, workspace, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -19,9 +19,11 @@ struct Problem {
   int32_t causal;
 };
 
-// Forward, bf16 tensors (tcgen05 path).  o [T,hq,d] bf16, lse [hq,T] f32.
+// Forward, bf16 tensors (tcgen05 path).  o [T,hq,d] bf16, lse [hq,T] f32; workspace:
+// kFwdWorkspaceBytes (the work-item counter).
+constexpr size_t kFwdWorkspaceBytes = 256;
 cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, const void* v, void* o,
-                            float* lse, cudaStream_t stream);
+                            float* lse, void* workspace, cudaStream_t stream);
 
 // Backward, bf16 tensors (tcgen05 path).  Workspace: bwd_bf16_workspace_bytes(pb).
 size_t bwd_bf16_workspace_bytes(const Problem& pb);

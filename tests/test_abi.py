@@ -61,6 +61,8 @@ def _fwd(lib, **kw):
     (dict(lse=None), attn.ATTN_ERR_INVALID_ARG),
     (dict(o=0x1008), attn.ATTN_ERR_INVALID_ARG),
     (dict(batch=-1, total=-8), attn.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None, wsb=0), attn.ATTN_ERR_INVALID_ARG),          # bf16 needs the 256-byte workspace
+    (dict(ws=0x1008, wsb=256), attn.ATTN_ERR_INVALID_ARG),      # misaligned workspace
 ])
 def test_fwd_rejects_bad_arguments_on_host(lib, kw, status):
     assert _fwd(lib, **kw) == status
@@ -83,7 +85,9 @@ def test_bwd_rejects_small_workspace(lib):
 
 
 def test_workspace_sizes(lib):
-    assert lib.attn_fwd_workspace_size(4, 2048, 8192, 16, 16, 128, 0) == 0
+    assert lib.attn_fwd_workspace_size(4, 2048, 8192, 16, 16, 128, 0) == 256   # the work-item counter
+    assert lib.attn_fwd_workspace_size(4, 2048, 8192, 16, 16, 128, 1) == 0     # fp32 check mode
+    assert lib.attn_fwd_workspace_size(0, 0, 0, 16, 16, 128, 0) == 0
     assert lib.attn_bwd_workspace_size(1, 0, 0, 4, 4, 64, 0) == 0
     assert lib.attn_bwd_workspace_size(2, 10, 20, 4, 2, 32, 1) == 4 * 20 * 4   # fp32 mode: D only
 
