@@ -42,6 +42,9 @@ def _bind(lib):
     lib.oracle_attn_bwd_ex.restype = ctypes.c_int
     lib.oracle_attn_probs.argtypes = [dp, dp, i32, i32, f64, i32, dp, dp]
     lib.oracle_attn_fwd_cross.argtypes = [dp, dp, dp, ip, ip, i32, i32, i32, i32, f64, i32, dp, dp, i32]
+    lib.oracle_attn_fwd_fp8sim.argtypes = [dp, dp, dp, ip, i32, i32, i32, i32, f64, i32, i32, dp, dp, i32]
+    lib.oracle_round_e4m3.argtypes = [f64]
+    lib.oracle_round_e4m3.restype = f64
     lib.oracle_attn_probs.restype = ctypes.c_int
     _lib = lib
 
@@ -138,6 +141,31 @@ def attn_fwd_cross(q, k, v, cu_q, cu_k, scale=None, causal=False, threads=None):
                                        threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_cross failed with code {rc}")
+    return o, lse
+
+
+def round_e4m3(x: float) -> float:
+    """x rounded to the nearest e4m3 value (ties to even), saturating at +-448."""
+    return float(_load().oracle_round_e4m3(float(x)))
+
+
+def attn_fwd_fp8sim(q, k, v, cu_seqlens=None, scale=None, causal=False, round_p=True, threads=None):
+    """The FP8 forward's steps on dequantised Q, K, V: blockwise online softmax (128-key
+    blocks, running max moved only past 8 log2 units) with the probabilities that
+    multiply V rounded to e4m3.  round_p=False is the exact forward."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    cu = _cu(cu_seqlens, T)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.full((T, hq, d), np.nan)
+    lse = np.full((hq, T), np.nan)
+    rc = _load().oracle_attn_fwd_fp8sim(_ptr(q), _ptr(k), _ptr(v), _ptr(cu, ctypes.c_int32), len(cu) - 1, hq, hkv, d,
+                                        float(scale), int(bool(causal)), int(bool(round_p)), _ptr(o), _ptr(lse),
+                                        threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_fp8sim failed with code {rc}")
     return o, lse
 
 

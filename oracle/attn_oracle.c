@@ -421,6 +421,143 @@ int oracle_attn_fwd_cross(const double *q, const double *k, const double *v,
     return W.failed ? ORACLE_NO_MEM : ORACLE_OK;
 }
 
+/* ---- FP8 forward: the steps of the quantised method -------------------------------
+ * The "Flash-Attention" concept page names FP8 attention (FlashAttention-3 on H100,
+ * 观察 2; quantised attention, 设计空间 路线 4) and conditional rescaling (已知局限)
+ * without a recipe, so this oracle follows the steps of the quantised forward rather than a
+ * closed form: Q, K, V are the dequantised e4m3 values (passed in as doubles); each row
+ * runs the online softmax of the "FlashAttention 与高效注意力内核" tutorial (sections
+ * Online Softmax 技巧 / 修正公式) over 128-key blocks, the running max moving only when a
+ * block's max exceeds it by more than 8 in log2 units, and the probabilities that multiply
+ * V are rounded to e4m3 (round to nearest even, saturating at 448) while the row sum l
+ * uses them unrounded:
+ *     m_new = max(m, blockmax) if blockmax > m + 8 else m        (log2 units)
+ *     p_j   = 2^(s_j log2 e - m_new),  l = l 2^(m - m_new) + sum_j p_j
+ *     O     = O 2^(m - m_new) + sum_j e4m3(p_j) v_j
+ * and finally O / l, LSE = m ln 2 + ln l.  With round_p = 0 this is the exact forward
+ * (the online softmax reaches the plain definition up to rounding). */
+double oracle_round_e4m3(double x)
+{
+    if (x != x) return x;
+    const double a = fabs(x);
+    if (a >= 448.0) return copysign(448.0, x);
+    double q;                                  /* spacing of e4m3 values around a */
+    if (a < 0.015625) {
+        q = 0.001953125;                       /* subnormals (and the lowest binade): 2^-9 */
+    } else {
+        int e;
+        (void)frexp(a, &e);                    /* a = f 2^e, f in [0.5, 1): 3 mantissa bits */
+        q = ldexp(1.0, e - 4);
+    }
+    const double r = nearbyint(a / q) * q;     /* default rounding mode: nearest, ties to even */
+    return copysign(r > 448.0 ? 448.0 : r, x);
+}
+
+typedef struct {
+    problem P;                  /* q, k, v (dequantised), hq, hkv, d, scale, causal, o, lse, cu */
+    int32_t round_p;
+    int64_t T;
+    int64_t next, nitems;       /* items: (sequence, query head) */
+    pthread_mutex_t lock;
+    int failed;
+} fp8_work;
+
+#define FP8_KEYS_PER_BLOCK 128
+#define FP8_RESCALE_SKIP 8.0
+
+static void *fp8_worker(void *arg)
+{
+    fp8_work *W = (fp8_work *)arg;
+    problem *P = &W->P;
+    int64_t maxn = 1;
+    for (int b = 0; b < P->nseq; ++b) {
+        const int64_t n = P->cu[b + 1] - P->cu[b];
+        if (n > maxn) maxn = n;
+    }
+    double *s = (double *)malloc((size_t)maxn * sizeof(double));
+    double *acc = (double *)malloc((size_t)P->d * sizeof(double));
+    if (!s || !acc) {
+        pthread_mutex_lock(&W->lock); W->failed = 1; pthread_mutex_unlock(&W->lock);
+        free(s); free(acc);
+        return NULL;
+    }
+    const double log2e = 1.4426950408889634, ln2 = 0.6931471805599453;
+    for (;;) {
+        pthread_mutex_lock(&W->lock);
+        const int64_t it = W->next++;
+        pthread_mutex_unlock(&W->lock);
+        if (it >= W->nitems) break;
+        const int b = (int)(it / P->hq);
+        const int h = (int)(it % P->hq);
+        const int g = (int)(((int64_t)h * P->hkv) / P->hq);
+        const int64_t t0 = P->cu[b];
+        const int n = (int)(P->cu[b + 1] - t0);
+        for (int i = 0; i < n; ++i) {
+            const int64_t row = t0 + i;
+            score_row(P, row, t0, n, visible_keys(i, n, P->causal), h, s);
+            double m = -INFINITY, l = 0.0;
+            for (int c = 0; c < P->d; ++c) acc[c] = 0.0;
+            for (int j0 = 0; j0 < n; j0 += FP8_KEYS_PER_BLOCK) {
+                const int j1 = j0 + FP8_KEYS_PER_BLOCK < n ? j0 + FP8_KEYS_PER_BLOCK : n;
+                double mx = -INFINITY;
+                for (int j = j0; j < j1; ++j) if (s[j] > mx) mx = s[j];
+                const double cand = mx * log2e;
+                const double m_new = cand > m + FP8_RESCALE_SKIP ? cand : m;
+                if (m_new == -INFINITY) continue;             /* nothing visible yet */
+                const double alpha = m == -INFINITY ? 0.0 : exp2(m - m_new);
+                l *= alpha;
+                for (int c = 0; c < P->d; ++c) acc[c] *= alpha;
+                for (int j = j0; j < j1; ++j) {
+                    if (s[j] == -INFINITY) continue;
+                    const double pj = exp2(s[j] * log2e - m_new);
+                    l += pj;
+                    const double pv = W->round_p ? oracle_round_e4m3(pj) : pj;
+                    const double *vj = P->v + ((t0 + j) * P->hkv + g) * P->d;
+                    for (int c = 0; c < P->d; ++c) acc[c] += pv * vj[c];
+                }
+                m = m_new;
+            }
+            double *oi = P->o + (row * P->hq + h) * P->d;
+            for (int c = 0; c < P->d; ++c) oi[c] = l > 0.0 ? acc[c] / l : 0.0;
+            P->lse[(int64_t)h * W->T + row] = l > 0.0 ? m * ln2 + log(l) : -INFINITY;
+        }
+    }
+    free(s);
+    free(acc);
+    return NULL;
+}
+
+int oracle_attn_fwd_fp8sim(const double *q, const double *k, const double *v,
+                           const int32_t *cu_seqlens, int32_t nseq,
+                           int32_t hq, int32_t hkv, int32_t d, double scale, int32_t causal,
+                           int32_t round_p, double *o, double *lse, int32_t nthreads)
+{
+    int rc = check_args(cu_seqlens, nseq, hq, hkv, d);
+    if (rc) return rc;
+    fp8_work W;
+    memset(&W, 0, sizeof W);
+    W.P.q = q; W.P.k = k; W.P.v = v; W.P.cu = cu_seqlens; W.P.nseq = nseq;
+    W.P.hq = hq; W.P.hkv = hkv; W.P.d = d; W.P.scale = scale; W.P.causal = causal;
+    W.P.o = o; W.P.lse = lse;
+    W.round_p = round_p;
+    W.T = cu_seqlens[nseq];
+    W.nitems = (int64_t)nseq * hq;
+    pthread_mutex_init(&W.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    pthread_t *tid = (pthread_t *)malloc((size_t)nthreads * sizeof(pthread_t));
+    int started = 0;
+    if (tid) {
+        for (; started < nthreads; ++started)
+            if (pthread_create(&tid[started], NULL, fp8_worker, &W) != 0) break;
+    }
+    if (started == 0) fp8_worker(&W);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    free(tid);
+    pthread_mutex_destroy(&W.lock);
+    return W.failed ? ORACLE_NO_MEM : ORACLE_OK;
+}
+
 /* Forward: o [T,hq,d], lse [hq,T].  row_sel (optional, [T]) restricts which rows are
  * written; other entries of o and lse are left untouched. */
 int oracle_attn_fwd(const double *q, const double *k, const double *v,

@@ -12,6 +12,7 @@ import pytest
 import oracle
 from tests import test_oracle as pins
 from tests import test_oracle_decode as dpins
+from tests import test_oracle_fp8 as fpins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
 
@@ -32,6 +33,9 @@ MUTANTS = {
                           "if (lse_in) lse[(int64_t)h * T + t] = lse[(int64_t)h * T + t];"),
     "given O ignored for D": ("dd[(int64_t)h * T + t] = dsum;", "(void)dsum;"),
     "score mask boundary off by one": ("if (j >= vis) { s[j] = -INFINITY; continue; }", "if (j > vis) { s[j] = -INFINITY; continue; }"),
+    "fp8 row sum from the rounded weights": ("                    l += pj;\n",
+                                            "                    l += W->round_p ? oracle_round_e4m3(pj) : pj;\n"),
+    "fp8 weights not rounded": ("const double pv = W->round_p ? oracle_round_e4m3(pj) : pj;", "const double pv = pj;"),
     "decode causal mask aligned top-left": ("const int v = lk - lq + i + 1;", "const int v = i + 1;"),
     "decode LSE stored to the sequence's first row": ("P->lse[(int64_t)h * W->tq + row] = lse;",
                                                       "P->lse[(int64_t)h * W->tq + q0] = lse;"),
@@ -58,6 +62,8 @@ def _battery():
         lambda: dpins.test_cross_matches_brute_force(([1, 3], [2, 6]), True),
         lambda: dpins.test_cross_matches_brute_force(([2, 3], [7, 3]), False),
         lambda: dpins.test_cross_zero_queries_average_the_visible_values(),
+        lambda: fpins.test_two_key_example_rounds_the_weights_but_not_the_sum(),
+        lambda: fpins.test_unrounded_steps_equal_the_exact_forward(True, 30.0),
     ]
     for c in checks:
         try:
