@@ -501,6 +501,182 @@ def run_decode(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------------------
+# FP8 (e4m3) forward: per-head quantised operands, both products on e4m3 tensor cores
+# ---------------------------------------------------------------------------------------
+FP8_METRIC = "FP8 (e4m3) attention forward TFLOPs/s on 1 B200 (d=128) and % of dense FP8 peak"
+FP8_WORKLOADS = {"fp8_mha2k": lambda: W.mha2k(False)}
+
+
+def fp8_config(n_gpus):
+    w = FP8_WORKLOADS[WORKLOAD]()
+    return {"workload": f"{WORKLOAD}: B={w.batch} Hq={w.hq} Hkv={w.hkv} N={w.seqlen} d={w.d}, e4m3 Q/K/V with "
+                        "per-head scales (quantised once, outside the timed step), forward only, non-causal and "
+                        "causal",
+            "global_batch": w.batch * n_gpus, "seq_len": w.seqlen, "heads": w.hq, "head_dim": w.d,
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{n_gpus}"}
+
+
+def fp8_oracle_sample(heads=None, budget_s=None):
+    """The oracle's FP8 forward (fp8sim) on whole heads of sequence 0, both masks, on the
+    operands dequantised from a per-head e4m3 quantisation done here on the CPU."""
+    import oracle
+    w = FP8_WORKLOADS[WORKLOAD]()
+    if "fp8" not in _ORACLE_CACHE:
+        q, k, v, _, _ = W.make_inputs(w, with_grad=False)
+        deq = []
+        for x in (q, k, v):
+            xf = x.float()
+            amax = xf.abs().amax(dim=(0, 2))
+            ds = torch.where(amax > 0, amax / torch.tensor(448.0), torch.ones_like(amax))
+            x8 = (xf / ds[None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn)
+            deq.append(x8.double() * ds.double()[None, :, None])
+        _ORACLE_CACHE["fp8"] = deq
+    q, k, v = _ORACLE_CACHE["fp8"]
+    n, G = w.seqlen, w.hq // w.hkv
+    threads = oracle.default_threads()
+    flops, secs, done = 0.0, 0.0, 0
+    for h in range(w.hq):
+        if (heads is not None and done >= heads) or (budget_s is not None and secs >= budget_s):
+            break
+        qs = q[:n, h:h + 1].numpy().copy()
+        ks, vs = (t[:n, h // G:h // G + 1].numpy().copy() for t in (k, v))
+        for causal in (False, True):
+            t0 = time.perf_counter()
+            oracle.attn_fwd_fp8sim(qs, ks, vs, scale=w.scale, causal=causal, threads=threads)
+            secs += time.perf_counter() - t0
+            flops += 4.0 * n * n * w.d * (0.5 if causal else 1.0)
+        done += 1
+    return flops, secs, done, threads
+
+
+def run_reference_fp8(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        fp8_oracle_sample(heads=1)
+    flops = secs = 0.0
+    threads = 1
+    for _ in range(args.steps):
+        f, s_, _, threads = fp8_oracle_sample(heads=1)
+        flops += f
+        secs += s_
+    value = flops / secs / 1e12
+    line = {"impl": "reference", "metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": fp8_config(world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"fp64 CPU oracle (FP8 steps), 1 head of sequence 0 of {WORKLOAD}, both "
+                                       "masks, per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_fp8(args, rank, world, local_rank):
+    import io_aware_exact_qk_b200 as attn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    attn.load_library()
+    w = dataclasses.replace(FP8_WORKLOADS[WORKLOAD](), seed=FP8_WORKLOADS[WORKLOAD]().seed + rank)
+    q, k, v, _, _ = W.make_inputs(w, with_grad=False)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    ops = attn.attn_fp8_quantize(qd, kd, vd, w.batch)
+    outs = {c: (torch.empty_like(qd), torch.empty(w.hq, w.total_tokens, device=dev)) for c in (False, True)}
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    variants = [w, w.with_causal(True)]
+
+    def step():
+        for c in (False, True):
+            attn.attn_fwd_fp8(*ops, batch=w.batch, scale=w.scale, causal=c, o=outs[c][0], lse=outs[c][1],
+                              workspace=ws)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    flops_step = sum(x.fwd_flops() for x in variants)
+    for _ in range(args.warmup):
+        step()
+    attn.attn_get_device_error()
+    barrier()
+    attn.attn_profile_collect()
+    attn.attn_profile_enable(True)
+    launches0 = attn.attn_launch_count()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        for s_, e_ in events:
+            flush.zero_()
+            s_.record(stream)
+            step()
+            e_.record(stream)
+        barrier()
+    attn.attn_profile_enable(False)
+    launches = attn.attn_launch_count() - launches0
+    per_kernel = attn.attn_profile_collect()
+    attn.attn_get_device_error()
+    total_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in events), world, dev)
+    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"quick": True, "value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
+                              "kernels": {k_: list(v_) for k_, v_ in per_kernel.items()}, "gpu_launches": launches}))
+        return
+    # end to end: bf16 Q, K, V from pinned host memory, quantised and attended on the
+    # device, O and LSE of both masks back to pinned host memory
+    hq_, hk_, hv_ = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    ho = {c: (torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory(),
+              torch.empty(w.hq, w.total_tokens).pin_memory()) for c in (False, True)}
+    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_))
+    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in ho.values())
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        qd.copy_(hq_, non_blocking=True)
+        kd.copy_(hk_, non_blocking=True)
+        vd.copy_(hv_, non_blocking=True)
+        ops = attn.attn_fp8_quantize(qd, kd, vd, w.batch)
+        step()
+        for c in (False, True):
+            ho[c][0].copy_(outs[c][0], non_blocking=True)
+            ho[c][1].copy_(outs[c][1], non_blocking=True)
+    e1.record(stream)
+    barrier()
+    attn.attn_get_device_error()
+    e2e_value = world * flops_step * args.steps / (max_over_ranks(e0.elapsed_time(e1), world, dev) / 1e3) / 1e12
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]     # dense e4m3 runs at twice the bf16 rate
+    dom = "fwd_fp8_sm100"
+    dom_ms, dom_n = per_kernel[dom]
+    achieved = flops_step * args.steps / (dom_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": fp8_peak, "unit": UNIT,
+                "frac": achieved / fp8_peak, "traffic": traffic_record(dom),
+                "peak_source": f"{peaks['source']} dense bf16 (burst) x 2, the nominal e4m3 / bf16 ratio",
+                "flops_per_launch": flops_step * args.steps / dom_n, "mean_launch_ms": dom_ms / dom_n}
+    breakdown = {k_: {"launches": n_, "total_ms": ms, "share": ms / sum(x[0] for x in per_kernel.values())}
+                 for k_, (ms, n_) in sorted(per_kernel.items())}
+    cpu = None
+    if world == 1:
+        f, s_, heads, threads = fp8_oracle_sample(budget_s=12.0)
+        cpu = {"value": f / s_ / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 CPU oracle (FP8 steps), {heads} whole head(s) of sequence 0 of {WORKLOAD}, both "
+                         f"masks, {s_:.1f} s"}
+    line = {"metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate, bf16 O)", "data": DATA,
+            "config": fp8_config(world), "pct_of_peak": value / fp8_peak, "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "clocks": clocks.summary(), "kernels": breakdown}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,7 +685,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha2k",
                     help="mha2k (the metric's configuration), sweep_d<d>_n<N>, gqa8k, varlen16, long32k; "
-                         "or a split-KV decode workload: decode8k, decode_var, decode_spec4")
+                         "or a split-KV decode workload: decode8k, decode_var, decode_spec4; "
+                         "or the FP8 forward: fp8_mha2k")
     ap.add_argument("--quick", action="store_true",
                     help="device timing only: skip the end-to-end loop and the CPU baseline (profiling runs)")
     args = ap.parse_args()
@@ -523,8 +700,9 @@ def main():
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
     decode = WORKLOAD in DECODE_WORKLOADS
+    fp8 = WORKLOAD in FP8_WORKLOADS
     if args.impl == "reference":
-        (run_reference_decode if decode else run_reference)(args, rank, world)
+        (run_reference_decode if decode else run_reference_fp8 if fp8 else run_reference)(args, rank, world)
         return
     if world > 1:
         import datetime
@@ -532,7 +710,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        (run_decode if decode else run_ours)(args, rank, world, local_rank)
+        (run_decode if decode else run_fp8 if fp8 else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -127,7 +127,8 @@ const char* kernel_kind_name(int kind) {
   static const char* names[K_NUM_KINDS] = {"fwd_bf16_sm100",  "bwd_preprocess",       "bwd_bf16_sm100",
                                            "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",
                                            "bwd_fp32_dkdv_kernel", "decode_bf16_sm100", "decode_combine",
-                                           "merge_partial",   "merge_finish"};
+                                           "merge_partial",   "merge_finish",         "fwd_fp8_sm100",
+                                           "fp8_quantize"};
   return (kind >= 0 && kind < K_NUM_KINDS) ? names[kind] : "";
 }
 
@@ -183,6 +184,21 @@ bool encode_tma_3d_box(void* tmap_out, const void* base, int d, int heads, int r
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tma_u8_3d(void* tmap_out, const void* base, int dim0, int dim1, int dim2, uint64_t stride1,
+                      uint64_t stride2, int box0, int box1, int box2) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
+  const cuuint64_t strides[2] = {(cuuint64_t)stride1, (cuuint64_t)stride2};
+  const cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, (cuuint32_t)box2};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(reinterpret_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_tma_3d_f32(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
@@ -200,6 +216,20 @@ bool encode_tma_3d_f32(void* tmap_out, const void* base, int d, int heads, int r
 }  // namespace attn
 
 using namespace attn;
+
+namespace {
+// Shapes of the FP8 calls: a fixed-length batch (batch sequences of seqlen tokens), d = 128.
+attn_status check_fp8(int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                      Problem* pb) {
+  if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 forward needs head dim 128 (got %d)", d);
+  if (batch < 0 || seqlen < 0) return fail(ATTN_ERR_INVALID_ARG, "negative batch / seqlen");
+  if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+  if ((int64_t)batch * hkv > 65535) return fail(ATTN_ERR_UNSUPPORTED, "batch * hkv must be <= 65535");
+  if ((int64_t)batch * hkv * d * fp8_vt_pitch(seqlen) > ((int64_t)1 << 40))
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+  return check_shapes(nullptr, batch, seqlen, seqlen, batch * seqlen, hq, hkv, d, scale, causal, ATTN_BF16, pb);
+}
+}  // namespace
 
 extern "C" {
 
@@ -227,6 +257,43 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t*
   return from_cuda(launch_fwd_fp32(pb, static_cast<const float*>(q), static_cast<const float*>(k),
                                    static_cast<const float*>(v), static_cast<float*>(o), lse, s),
                    "attn_fwd (fp32 check mode) launch");
+}
+
+attn_status attn_fp8_quantize(const void* q, const void* k, const void* v, int32_t batch, int32_t seqlen, int32_t hq,
+                              int32_t hkv, int32_t d, void* q8, void* k8, void* vt8, float* descale_q,
+                              float* descale_k, float* descale_v, void* stream) {
+  Problem pb;
+  attn_status st = check_fp8(batch, seqlen, hq, hkv, d, 1.f, 0, &pb);
+  if (st != ATTN_OK) return st;
+  if (batch == 0 || seqlen == 0) return ok();
+  if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) || (st = check_ptr(q8, "q8")) ||
+      (st = check_ptr(k8, "k8")) || (st = check_ptr(vt8, "vt8")) || (st = check_ptr(descale_q, "descale_q")) ||
+      (st = check_ptr(descale_k, "descale_k")) || (st = check_ptr(descale_v, "descale_v")))
+    return st;
+  return from_cuda(launch_fp8_quantize(q, k, v, batch, seqlen, hq, hkv, d, q8, k8, vt8, descale_q, descale_k,
+                                       descale_v, static_cast<cudaStream_t>(stream)),
+                   "attn_fp8_quantize launch");
+}
+
+attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* descale_q,
+                         const float* descale_k, const float* descale_v, int32_t batch, int32_t seqlen, int32_t hq,
+                         int32_t hkv, int32_t d, float scale, int32_t causal, void* o, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Problem pb;
+  attn_status st = check_fp8(batch, seqlen, hq, hkv, d, scale, causal, &pb);
+  if (st != ATTN_OK) return st;
+  if (batch == 0 || seqlen == 0) return ok();
+  if ((st = check_ptr(q8, "q8")) || (st = check_ptr(k8, "k8")) || (st = check_ptr(vt8, "vt8")) ||
+      (st = check_ptr(descale_q, "descale_q")) || (st = check_ptr(descale_k, "descale_k")) ||
+      (st = check_ptr(descale_v, "descale_v")) || (st = check_ptr(o, "o")) || (st = check_ptr(lse, "lse")))
+    return st;
+  if (workspace_bytes < kFwdWorkspaceBytes)
+    return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes,
+                kFwdWorkspaceBytes);
+  if ((st = check_ptr(workspace, "workspace"))) return st;
+  return from_cuda(launch_fwd_fp8(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace,
+                                  static_cast<cudaStream_t>(stream)),
+                   "attn_fwd_fp8 launch");
 }
 
 }  // extern "C"

@@ -1,0 +1,149 @@
+// fp8_quant.cu -- e4m3 operands for the FP8 forward.
+//
+// The "Flash-Attention" concept page names FP8 attention (FlashAttention-3 on H100,
+// 观察 2; quantised attention with its scaling strategies, 设计空间 路线 4).  The scaling
+// here is per head: descale_x[h] = amax_h / 448 (448 = the largest e4m3 value), and
+// x8 = e4m3(x / descale_x[h]) (fp32 division, then rounded to nearest even with
+// saturation).  Q and K keep their [T, heads, d] layout; V is written transposed per
+// (sequence, head), vt8 [batch * hkv][d][pitch] (tokens contiguous, pitch = seqlen rounded
+// up to 16, zero-padded), the K-major B operand of the P V product.
+#include <algorithm>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr float kE4m3Max = 448.f;
+
+__device__ __forceinline__ uint8_t to_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x), "f"(x));   // x in both bytes
+  return (uint8_t)(r & 0xFFu);
+}
+
+// amax over |x| per head of a [T, heads, d] bf16 tensor, as float bits (non-negative floats
+// order like their bit patterns) into amax_bits[heads] (zeroed beforehand).
+__global__ void __launch_bounds__(256) amax_per_head(const __nv_bfloat16* __restrict__ x, int64_t n, int heads, int d,
+                                                     unsigned* __restrict__ amax_bits) {
+  // one block-stride walk over 8-element groups; each group lies inside one (token, head)
+  const int64_t n8 = n / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    const int head = (int)((i * 8 / d) % heads);
+    atomicMax(amax_bits + head, __float_as_uint(m));
+  }
+}
+
+__global__ void amax_to_descale(unsigned* __restrict__ bits, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float a = __uint_as_float(bits[i]);
+    const float ds = a > 0.f ? a / kE4m3Max : 1.f;
+    reinterpret_cast<float*>(bits)[i] = ds;
+  }
+}
+
+// x8[t][h][c] = e4m3(x[t][h][c] / descale[h]), 8 elements per thread.
+__global__ void __launch_bounds__(256) quantize_rows(const __nv_bfloat16* __restrict__ x, int64_t n, int heads, int d,
+                                                     const float* __restrict__ descale, uint8_t* __restrict__ x8) {
+  const int64_t n8 = n / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    const float ds = descale[(int)((i * 8 / d) % heads)];
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      const uint32_t pair = (uint32_t)to_e4m3(__fdiv_rn(f.x, ds)) | ((uint32_t)to_e4m3(__fdiv_rn(f.y, ds)) << 8);
+      if (e < 2) lo |= pair << (16 * e);
+      else hi |= pair << (16 * (e - 2));
+    }
+    reinterpret_cast<uint2*>(x8)[i] = make_uint2(lo, hi);
+  }
+}
+
+// vt8[b * hkv + g][c][t] = e4m3(v[b * seqlen + t][g][c] / descale[g]) for t < seqlen and 0
+// for seqlen <= t < pitch, through a 64-token x 64-feature shared tile so that both the
+// reads (along c) and the writes (along t) are coalesced.
+__global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16* __restrict__ v, int seqlen,
+                                                             int pitch, int hkv, int d, const float* __restrict__ descale,
+                                                             uint8_t* __restrict__ vt8) {
+  __shared__ uint8_t tile[64][64 + 4];
+  const int z = blockIdx.z;   // b * hkv + g
+  const int g = z % hkv, b = z / hkv;
+  const int c0 = blockIdx.y * 64;
+  const int t0 = blockIdx.x * 64;
+  const float ds = descale[g];
+  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
+    const int tt = e / 64, cc = e % 64;
+    const int t = t0 + tt;
+    float x = 0.f;
+    if (t < seqlen) x = __bfloat162float(v[(((size_t)b * seqlen + t) * hkv + g) * d + c0 + cc]);
+    tile[cc][tt] = to_e4m3(__fdiv_rn(x, ds));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
+    const int cc = e / 64, tt = e % 64;
+    const int t = t0 + tt;
+    if (t < pitch) vt8[((size_t)z * d + c0 + cc) * pitch + t] = tile[cc][tt];
+  }
+}
+
+int q8_sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int batch, int seqlen, int hq, int hkv,
+                                int d, void* q8, void* k8, void* vt8, float* descale_q, float* descale_k,
+                                float* descale_v, cudaStream_t stream) {
+  const int total_tokens = batch * seqlen;
+  if (total_tokens == 0 || d % 64 != 0) return total_tokens == 0 ? cudaSuccess : cudaErrorInvalidValue;
+  const int pitch = fp8_vt_pitch(seqlen);
+  const int grid = q8_sm_count() * 8;
+  const int64_t nq = (int64_t)total_tokens * hq * d, nk = (int64_t)total_tokens * hkv * d;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(descale_q, 0, hq * sizeof(float), stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(descale_k, 0, hkv * sizeof(float), stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(descale_v, 0, hkv * sizeof(float), stream)) != cudaSuccess) return e;
+  {
+    LaunchScope scope(K_FP8_QUANTIZE, stream);
+    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), nq, hq, d,
+                                           reinterpret_cast<unsigned*>(descale_q));
+    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), nk, hkv, d,
+                                           reinterpret_cast<unsigned*>(descale_k));
+    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), nk, hkv, d,
+                                           reinterpret_cast<unsigned*>(descale_v));
+    amax_to_descale<<<(hq + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_q), hq);
+    amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_k), hkv);
+    amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_v), hkv);
+    quantize_rows<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), nq, hq, d, descale_q,
+                                           static_cast<uint8_t*>(q8));
+    quantize_rows<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), nk, hkv, d, descale_k,
+                                           static_cast<uint8_t*>(k8));
+    quantize_v_transposed<<<dim3((pitch + 63) / 64, d / 64, batch * hkv), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(v), seqlen, pitch, hkv, d, descale_v, static_cast<uint8_t*>(vt8));
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace attn

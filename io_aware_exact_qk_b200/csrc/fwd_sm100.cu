@@ -58,17 +58,22 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
 constexpr int kItemSlots = 4;  // ring of work-item indices the producer hands to the other roles
 
-template <int D>
+// FP8: Q, K and V^T (per-head transposed V) are e4m3 tiles and both products run as
+// kind::f8f6f4 with 32-element K steps; P goes to TMEM as four e4m3 per column.
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int SW = D >= 64 ? 128 : 64;    // swizzle span == SMEM row pitch (bytes)
-  static constexpr int PANEL = SW / 2;             // bf16 elements per panel row
+  static constexpr int ELEM = FP8 ? 1 : 2;         // bytes per Q/K/V element
+  static constexpr int SW = (FP8 || D >= 64) ? 128 : 64;   // swizzle span == SMEM row pitch (bytes)
+  static constexpr int PANEL = SW / ELEM;          // elements per panel row
   static constexpr int NPANEL = D / PANEL;         // panels per tile
   static constexpr int PANEL_BYTES = kRows * SW;   // one panel of a 128-row tile
-  static constexpr int TILE_BYTES = kRows * D * 2;
-  static constexpr int STAGES = D == 128 ? 2 : (D == 64 ? 3 : 4);
+  static constexpr int TILE_BYTES = kRows * D * ELEM;
+  static constexpr int STAGES = FP8 ? 4 : (D == 128 ? 2 : (D == 64 ? 3 : 4));
   static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;   // descriptor swizzle code
   static constexpr int SBO = 8 * SW;               // bytes between 8-row swizzle atoms
-  static constexpr int KSTEPS_PER_PANEL = SW / 32; // 16-element K steps inside one panel
+  static constexpr int KSTEPS_PER_PANEL = SW / 32; // 32-byte K steps inside one panel
+  static constexpr int S_KSTEPS = D * ELEM / 32;   // K steps of Q K^T
+  static constexpr int PV_KSTEPS = kKeys * ELEM / 32;   // K steps of P V (8 P columns each)
   // barrier slots
   static constexpr int B_QFULL = 0;
   static constexpr int B_QEMPTY = 1;
@@ -104,6 +109,9 @@ struct FwdParams {
   int32_t causal;
   __nv_bfloat16* o;
   float* lse;
+  const float* descale_q;    // FP8: per query head
+  const float* descale_k;    // FP8: per kv head
+  const float* descale_v;    // FP8: per kv head
   int32_t heads_per_group;   // causal order: (head, sequence) pairs whose K / V fit in L2
   int* item_counter;         // next unclaimed item (zeroed before the launch)
 };
@@ -160,11 +168,10 @@ __device__ __forceinline__ Item item_from(const FwdParams& p, int idx) {
   return it;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D>;
+template <int D, bool FP8>
+__device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                         const FwdParams& p) {
+  using C = FwdCfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);   // 1024-aligned (swizzle atoms)
@@ -256,9 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         it.seq_start + j * kKeys);
           if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
-          for (int pn = 0; pn < C::NPANEL; ++pn)
-            tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, hk,
-                        it.seq_start + j * kKeys);
+          if constexpr (FP8) {
+            // V^T [batch * hkv][d][padded seqlen]: a (128 keys) x (d rows) box, keys
+            // contiguous (K-major B); the key coordinate is a multiple of 128
+            tma_load_3d(sV + s * C::TILE_BYTES, &tmV, bar(C::B_VFULL + s), j * kKeys, 0, it.b * p.hkv + hk);
+          } else {
+            for (int pn = 0; pn < C::NPANEL; ++pn)
+              tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, hk,
+                          it.seq_start + j * kKeys);
+          }
         }
         ++qi;
       }
@@ -266,31 +279,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(kRows, kKeys, false, false);  // Q, K both K-major
-      const uint32_t idesc_pv = idesc_bf16_f32(kRows, D, false, true);       // V is MN-major (d contiguous)
+      // Q, K both K-major; V is MN-major in bf16 (d contiguous), V^T K-major in FP8
+      const uint32_t idesc_qk = FP8 ? idesc_e4m3_f32(kRows, kKeys, false, false)
+                                    : idesc_bf16_f32(kRows, kKeys, false, false);
+      const uint32_t idesc_pv = FP8 ? idesc_e4m3_f32(kRows, D, false, false) : idesc_bf16_f32(kRows, D, false, true);
       // Operand descriptors: bases computed once, advanced by compile-time offsets per
       // MMA (and by the tile/stage index per call), so one MMA issues in a few
       // instructions -- this single thread's issue rate bounds the tensor core.
       const uint64_t q_desc = smem_desc(sQ, 16, C::SBO, C::SWZ);
       const uint64_t k_desc = smem_desc(sK, 16, C::SBO, C::SWZ);
-      const uint64_t v_desc = smem_desc(sV, C::PANEL_BYTES, C::SBO, C::SWZ);
+      const uint64_t v_desc = FP8 ? smem_desc(sV, 16, C::SBO, C::SWZ) : smem_desc(sV, C::PANEL_BYTES, C::SBO, C::SWZ);
       auto issue_qk = [&](int t, int s) {
         const uint32_t d_tmem = tmem + t * kKeys;
         const uint64_t a0 = desc_advance(q_desc, (uint32_t)t * C::TILE_BYTES);
         const uint64_t b0 = desc_advance(k_desc, (uint32_t)s * C::TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
           const uint32_t off = (kk / C::KSTEPS_PER_PANEL) * C::PANEL_BYTES + (kk % C::KSTEPS_PER_PANEL) * 32;
-          mma_ss(d_tmem, desc_advance(a0, off), desc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (FP8)
+            mma_ss_f8(d_tmem, desc_advance(a0, off), desc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(d_tmem, desc_advance(a0, off), desc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int s, bool accumulate) {
         const uint32_t d_tmem = tmem + 2 * kKeys + t * D;
         const uint64_t b0 = desc_advance(v_desc, (uint32_t)s * C::TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint32_t a_tmem = tmem + t * kKeys + kk * 8;   // 16 bf16 keys = 8 packed columns
-          mma_ts(d_tmem, a_tmem, desc_advance(b0, kk * 16 * C::SW), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
+          const uint32_t a_tmem = tmem + t * kKeys + kk * 8;   // 8 packed columns: 16 bf16 / 32 e4m3 keys
+          if constexpr (FP8)
+            mma_ts_f8(d_tmem, a_tmem, desc_advance(b0, kk * 32), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(d_tmem, a_tmem, desc_advance(b0, kk * 16 * C::SW), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       uint32_t kv = 0, qi = 0;
@@ -358,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane_base = (warp & 3) * 32;          // TMEM lanes this warp may touch
     const uint32_t tS = tmem + ((uint32_t)lane_base << 16) + t * kKeys;
     const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + 2 * kKeys + t * D;
-    const float sl2 = p.scale_log2;
+    const float sl2_base = p.scale_log2;
     uint32_t sc = 0, oc = 0;   // S_t tiles and items consumed by this warpgroup
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -368,6 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_t = it.n[t];
       if (n_t == 0) continue;
       const int qi = it.q0 + t * kRows + lane_base + lane;   // query index inside the sequence
+      // FP8: the e4m3 products carry the per-head scales of Q and K
+      const int hk = it.h / (p.hq / p.hkv);
+      const float sl2 = FP8 ? sl2_base * p.descale_q[it.h] * p.descale_k[hk] : sl2_base;
       float m_used = -INFINITY;   // running max in log2 units (possibly stale by < 8)
       float mx_used = 0.f;        // the raw score maximum that m_used was formed from
       float l = 0.f;              // running sum of exp2(x - m_used)
@@ -418,7 +442,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx_used = mx;
         }
         const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
+        // P as bf16 pairs (64 columns) or, FP8, e4m3 quads (32 columns); key 2c, 2c+1 -> pair c
         uint32_t pk[64];
+        auto put_p = [&](uint32_t (&w)[64], int c, float p0, float p1) {
+          if constexpr (FP8) {
+            const uint32_t h = pack_e4m3x2(p0, p1);
+            if (c & 1) w[c >> 1] |= h << 16;
+            else w[c >> 1] = h;
+          } else {
+            w[c] = pack_bf16x2(p0, p1);
+          }
+        };
         const uint64_t sl2x2 = f2(sl2, sl2);
         const uint64_t negm = f2(-m_sub, -m_sub);
         uint64_t sum2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // 8 partial sums
@@ -430,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sl2x2, negm), x0, x1);
             const float p0 = ex2(x0), p1 = ex2(x1);
             sum2[c & 3] = add2(sum2[c & 3], f2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
+            put_p(pk, c, p0, p1);
           }
         } else {
           // A share of the exponentials (the pairs c with bit c % 8 set in kEmuPairs) runs
@@ -449,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               p1 = ex2(x1);
             }
             sum2[c & 3] = add2(sum2[c & 3], f2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
+            put_p(pk, c, p0, p1);
           }
         }
         float sum_lo, sum_hi;
@@ -457,9 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float rowsum = sum_lo + sum_hi;
         {
           uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
           tmem_st32(tS + 0, lo);
-          tmem_st32(tS + 32, hi);
+          if constexpr (!FP8) {
+            uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+            tmem_st32(tS + 32, hi);
+          }
         }
         float alpha = 1.f;
         if (m_new != m_used) {
@@ -492,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar(C::B_OFINAL + t), oc & 1, abort_flag)) { ok = false; break; }
       ++oc;
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f ? 1.f / l : 0.f) * (FP8 ? p.descale_v[hk] : 1.f);
       const bool row_ok = qi < it.len;
       // O / l as bf16, written through this warp's staging slice so that each store
       // instruction covers whole 128-byte row segments (a thread-per-row store would touch
@@ -539,9 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // LSE = m ln 2 + ln l, evaluated in double from the exact fp32 values the
         // exponentials used (m_used, l), minus the first-order effect of scale_log2 being
         // rounded to fp32 (exact when one score dominates the row), then rounded once.
+        // the rounding of the fp32 score factor (for FP8 it includes the two descales)
+        double skew = p.lse_skew;
+        if constexpr (FP8)
+          skew = (double)sl2 * 0.6931471805599453 -
+                 ((double)p.scale_log2 * 0.6931471805599453 - p.lse_skew) * p.descale_q[it.h] * p.descale_k[hk];
         float lse = -INFINITY;
         if (l > 0.f)
-          lse = (float)((double)m_used * 0.6931471805599453 + log((double)l) - p.lse_skew * (double)mx_used);
+          lse = (float)((double)m_used * 0.6931471805599453 + log((double)l) - skew * (double)mx_used);
         p.lse[(size_t)it.h * p.total_tokens + it.seq_start + qi] = lse;
       }
     }
@@ -555,6 +596,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  fwd_body<D, false>(tmQ, tmK, tmV, p);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_fp8_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmVt, const FwdParams p) {
+  fwd_body<D, true>(tmQ, tmK, tmVt, p);
+}
+
 int sm_count_fwd() {
   static int n = 0;
   if (n == 0) {
@@ -563,6 +618,48 @@ int sm_count_fwd() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
   }
   return n;
+}
+
+// Parameters and schedule shared by the bf16 and FP8 launches.
+template <int D, bool FP8>
+FwdParams fwd_params(const Problem& pb, void* o, float* lse, void* workspace) {
+  FwdParams p{};
+  p.cu_seqlens = pb.cu_seqlens;
+  p.seqlen = pb.seqlen;
+  p.max_seqlen = pb.max_seqlen;
+  p.total_tokens = pb.total_tokens;
+  p.hq = pb.hq;
+  p.hkv = pb.hkv;
+  p.batch = pb.batch;
+  p.n_pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
+  const int64_t items = (int64_t)p.n_pairs * pb.hq * pb.batch;
+  p.n_items = items > INT32_MAX ? -1 : (int)items;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.lse_skew = (double)p.scale_log2 * 0.6931471805599453 - (double)pb.scale;
+  p.causal = pb.causal;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  // causal order: (head, sequence) pairs whose K and V together stay within ~32 MB of L2
+  const int64_t kv_bytes = (int64_t)pb.max_seqlen * D * FwdCfg<D, FP8>::ELEM * 2;
+  p.heads_per_group = (int)std::max<int64_t>(
+      1, std::min<int64_t>((int64_t)pb.hq * pb.batch, (32ll << 20) / std::max<int64_t>(kv_bytes, 1)));
+  p.item_counter = static_cast<int*>(workspace);
+  return p;
+}
+
+template <int D, bool FP8, typename Kernel>
+cudaError_t launch_fwd_common(Kernel kernel, int kind, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
+  using C = FwdCfg<D, FP8>;
+  if (p.n_items < 0) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(p.item_counter, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(p.n_items, sm_count_fwd());
+  LaunchScope scope(kind, stream);
+  kernel<<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
 }
 
 template <int D>
@@ -574,36 +671,8 @@ cudaError_t launch_fwd_d(const Problem& pb, const void* q, const void* k, const 
       !encode_tma_3d(&tk, k, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys) ||
       !encode_tma_3d(&tv, v, D, pb.hkv, pb.total_tokens, C::PANEL, kKeys))
     return cudaErrorInvalidValue;
-  FwdParams p;
-  p.cu_seqlens = pb.cu_seqlens;
-  p.seqlen = pb.seqlen;
-  p.max_seqlen = pb.max_seqlen;
-  p.total_tokens = pb.total_tokens;
-  p.hq = pb.hq;
-  p.hkv = pb.hkv;
-  p.batch = pb.batch;
-  p.n_pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
-  const int64_t items = (int64_t)p.n_pairs * pb.hq * pb.batch;
-  if (items > INT32_MAX) return cudaErrorInvalidValue;
-  p.n_items = (int)items;
-  p.scale_log2 = pb.scale * kLog2e;
-  p.lse_skew = (double)p.scale_log2 * 0.6931471805599453 - (double)pb.scale;
-  p.causal = pb.causal;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  // causal order: (head, sequence) pairs whose K and V together stay within ~32 MB of L2
-  const int64_t kv_bytes = (int64_t)pb.max_seqlen * D * 2 * 2;
-  p.heads_per_group = (int)std::max<int64_t>(
-      1, std::min<int64_t>((int64_t)pb.hq * pb.batch, (32ll << 20) / std::max<int64_t>(kv_bytes, 1)));
-  p.item_counter = static_cast<int*>(workspace);
-  cudaError_t e = cudaMemsetAsync(p.item_counter, 0, sizeof(int), stream);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(fwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int grid = (int)std::min<int64_t>(items, sm_count_fwd());
-  LaunchScope scope(K_FWD_BF16, stream);
-  fwd_bf16_sm100<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  const FwdParams p = fwd_params<D, false>(pb, o, lse, workspace);
+  return launch_fwd_common<D, false>(fwd_bf16_sm100<D>, K_FWD_BF16, tq, tk, tv, p, stream);
 }
 
 }  // namespace
@@ -617,6 +686,27 @@ cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, con
     case 128: return launch_fwd_d<128>(pb, q, k, v, o, lse, workspace, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, const void* vt8,
+                           const float* descale_q, const float* descale_k, const float* descale_v, void* o,
+                           float* lse, void* workspace, cudaStream_t stream) {
+  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
+  if (pb.d != 128 || pb.cu_seqlens != nullptr) return cudaErrorInvalidValue;
+  constexpr int D = 128;
+  const int sp = fp8_vt_pitch(pb.seqlen);
+  alignas(64) CUtensorMap tq, tk, tv;
+  // Q8, K8: [tokens, heads, 128] bytes, one 128-byte swizzled row per token
+  if (!encode_tma_u8_3d(&tq, q8, D, pb.hq, pb.total_tokens, (uint64_t)D, (uint64_t)pb.hq * D, D, 1, kRows) ||
+      !encode_tma_u8_3d(&tk, k8, D, pb.hkv, pb.total_tokens, (uint64_t)D, (uint64_t)pb.hkv * D, D, 1, kKeys) ||
+      // V^T: [batch * hkv][128][sp] bytes, boxes of 128 keys x 128 features
+      !encode_tma_u8_3d(&tv, vt8, sp, D, pb.batch * pb.hkv, (uint64_t)sp, (uint64_t)D * sp, kKeys, D, 1))
+    return cudaErrorInvalidValue;
+  FwdParams p = fwd_params<D, true>(pb, o, lse, workspace);
+  p.descale_q = descale_q;
+  p.descale_k = descale_k;
+  p.descale_v = descale_v;
+  return launch_fwd_common<D, true>(fwd_fp8_sm100<D>, K_FWD_FP8, tq, tk, tv, p, stream);
 }
 
 }  // namespace attn

@@ -135,3 +135,25 @@ def test_decode_workspace_sizes(lib):
     # more splits than key tiles are clamped: 300 keys = 3 tiles
     assert lib.attn_fwd_decode_workspace_size(2, 1, 300, 2, 600, 8, 2, 64, 1, 16) == \
         ((3 * 2 * 8 * 64 * 4 + 255) // 256) * 256 + 3 * 8 * 2 * 4
+
+
+def _fwd_fp8(lib, d=128, batch=1, seqlen=64, hq=2, hkv=2, ptr=0x1000, o=0x1000, ws=0x1000, wsb=256, causal=0):
+    vp = ctypes.c_void_p
+    return lib.attn_fwd_fp8(vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), batch, seqlen, hq, hkv, d,
+                            ctypes.c_float(0.1), causal, vp(o), vp(ptr), vp(ws), wsb, None)
+
+
+def test_fp8_calls_reject_bad_arguments_on_host(lib):
+    assert _fwd_fp8(lib, d=64) == attn.ATTN_ERR_UNSUPPORTED            # e4m3 path is d = 128 only
+    assert _fwd_fp8(lib, ptr=None) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8(lib, o=0x1008) == attn.ATTN_ERR_INVALID_ARG         # misaligned output
+    assert _fwd_fp8(lib, wsb=0) == attn.ATTN_ERR_INVALID_ARG            # needs the 256-byte counter
+    assert _fwd_fp8(lib, hq=3, hkv=2) == attn.ATTN_ERR_UNSUPPORTED
+    assert _fwd_fp8(lib, causal=2) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8(lib, batch=0, ptr=None, o=None, ws=None, wsb=0) == attn.ATTN_OK   # empty: no-op
+    vp = ctypes.c_void_p
+    p = vp(0x1000)
+    assert lib.attn_fp8_quantize(p, p, p, 1, 64, 2, 2, 32, p, p, p, p, p, p, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fp8_quantize(p, p, p, 1, 64, 2, 2, 128, p, None, p, p, p, p, None) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fp8_quantize(None, None, None, 0, 64, 2, 2, 128, None, None, None, None, None, None,
+                                 None) == attn.ATTN_OK

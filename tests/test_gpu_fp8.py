@@ -1,0 +1,177 @@
+"""Parity of the FP8 (e4m3) forward with the fp64 oracle.
+
+Two calls are under test, both through the C ABI:
+
+* ``attn_fp8_quantize`` must reproduce, byte for byte, the per-head quantisation that this
+  file states on the CPU: descale = amax / 448 in fp32, x8 = e4m3(x / descale) with an
+  fp32 division and round-to-nearest-even (torch's float8_e4m3fn conversion, which
+  ``test_oracle_fp8`` pins to the oracle's rounding).  V goes out transposed per
+  (sequence, kv head) with a zero-padded token pitch.
+* ``attn_fwd_fp8`` runs on operands quantised here on the CPU (never on the GPU's own
+  quantisation), and ``oracle.attn_fwd_fp8sim`` runs on the same operands dequantised to
+  fp64.  The oracle takes the kernel's steps (128-key blocks, running max moved only past
+  8 log2 units, probabilities rounded to e4m3 before they multiply V), so the two agree
+  to the forward's bf16 tolerances (max |O - O_ref| <= 2e-2, rel-L2(O) <= 5e-3,
+  max |LSE - LSE_ref| <= 1e-3).  Against the exact forward of the dequantised operands
+  the probability rounding alone leaves a few 1e-2 of relative error, bounded below.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attn_workloads as W
+import io_aware_exact_qk_b200 as attn
+import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+E4M3_MAX = 448.0
+# rel-L2 of O against the exact forward of the dequantised operands: P rounded to e4m3
+# has a relative error of at most 2^-4 per entry, about 2^-6 in root-mean-square.
+FP8_EXACT_REL_L2 = 3e-2
+
+
+def pitch_of(seqlen):
+    return (seqlen + 15) // 16 * 16
+
+
+def quantize_cpu(x, heads):
+    """x [T, heads, d] bf16 -> (e4m3 bytes [T, heads, d] uint8, descale [heads] float32)."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=(0, 2))                                    # exact: bf16 values
+    ds = torch.where(amax > 0, amax / torch.tensor(E4M3_MAX, dtype=torch.float32), torch.ones_like(amax))
+    y = (xf / ds[None, :, None]).clamp(-E4M3_MAX, E4M3_MAX)            # fp32 division
+    x8 = y.to(torch.float8_e4m3fn).view(torch.uint8)
+    return x8, ds
+
+
+def transpose_v_cpu(v8, batch, seqlen):
+    """v8 [B S, hkv, d] -> [B hkv, d, pitch] with zero padding."""
+    T, hkv, d = v8.shape
+    out = torch.zeros(batch * hkv, d, pitch_of(seqlen), dtype=torch.uint8)
+    out[:, :, :seqlen] = v8.view(batch, seqlen, hkv, d).permute(0, 2, 3, 1).reshape(batch * hkv, d, seqlen)
+    return out
+
+
+def dequant(x8, ds):
+    return x8.view(torch.float8_e4m3fn).double() * ds.double()[None, :, None]
+
+
+def fp8_case(name, batch, seqlen, hq, hkv, causal, seed, qk_mult=1.0):
+    w = W.custom(name, [seqlen] * batch, hq, hkv, 128, causal, seed, qk_mult=qk_mult)
+    q, k, v, _, _ = W.make_inputs(w, with_grad=False)
+    return w, q, k, v
+
+
+CASES = [
+    # name, batch, seqlen, hq, hkv, causal, seed
+    ("fp8-1000-gqa", 2, 1000, 4, 2, False, 11),
+    ("fp8-1000-gqa-causal", 2, 1000, 4, 2, True, 12),
+    ("fp8-257", 1, 257, 2, 2, False, 13),
+    ("fp8-257-causal", 1, 257, 2, 1, True, 14),
+    ("fp8-2048-causal", 1, 2048, 2, 2, True, 15),
+    ("fp8-77", 3, 77, 2, 1, False, 16),
+]
+
+
+def run_fwd(w, q8, k8, vt8, dq, dk, dv):
+    dev = torch.device("cuda")
+    o, lse = attn.attn_fwd_fp8(q8.to(dev), k8.to(dev), vt8.to(dev), dq.to(dev), dk.to(dev), dv.to(dev),
+                               batch=w.batch, scale=w.scale, causal=w.causal)
+    attn.attn_get_device_error()
+    return parity.to_np(o), parity.to_np(lse)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_fp8_quantize_bit_exact(case):
+    name, batch, seqlen, hq, hkv, causal, seed = case
+    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed)
+    dev = torch.device("cuda")
+    q8, k8, vt8, dq, dk, dv = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), batch)
+    attn.attn_get_device_error()
+    q8_ref, dq_ref = quantize_cpu(q, hq)
+    k8_ref, dk_ref = quantize_cpu(k, hkv)
+    v8_ref, dv_ref = quantize_cpu(v, hkv)
+    assert torch.equal(dq.cpu(), dq_ref) and torch.equal(dk.cpu(), dk_ref) and torch.equal(dv.cpu(), dv_ref)
+    assert torch.equal(q8.cpu(), q8_ref)
+    assert torch.equal(k8.cpu(), k8_ref)
+    assert tuple(vt8.shape) == (batch * hkv, 128, pitch_of(seqlen))
+    assert torch.equal(vt8.cpu(), transpose_v_cpu(v8_ref, batch, seqlen))
+
+
+def test_fp8_quantize_zero_head_and_outlier_head():
+    """An all-zero head gets descale 1 and zero bytes; a head 300x larger gets its own scale."""
+    batch, seqlen, hq, hkv = 1, 200, 3, 3
+    w, q, k, v = fp8_case("fp8-heads", batch, seqlen, hq, hkv, False, 21)
+    q[:, 0] = 0
+    k[:, 2] *= 300
+    dev = torch.device("cuda")
+    q8, k8, vt8, dq, dk, dv = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), batch)
+    attn.attn_get_device_error()
+    assert float(dq[0]) == 1.0 and int(q8[:, 0].abs().sum()) == 0
+    k8_ref, dk_ref = quantize_cpu(k, hkv)
+    assert torch.equal(dk.cpu(), dk_ref) and torch.equal(k8.cpu(), k8_ref)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_fp8_forward_matches_oracle(case):
+    name, batch, seqlen, hq, hkv, causal, seed = case
+    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed)
+    q8, dq = quantize_cpu(q, hq)
+    k8, dk = quantize_cpu(k, hkv)
+    v8, dv = quantize_cpu(v, hkv)
+    vt8 = transpose_v_cpu(v8, batch, seqlen)
+    o, lse = run_fwd(w, q8, k8, vt8, dq, dk, dv)
+    qd, kd, vd = dequant(q8, dq).numpy(), dequant(k8, dk).numpy(), dequant(v8, dv).numpy()
+    cu = w.cu_seqlens().numpy()
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd, kd, vd, cu, scale=w.scale, causal=causal)
+    parity.check_fwd_bf16(o, lse, o_ref, lse_ref, tag=name)
+    # the approximation itself: against the exact forward of the same operands
+    o_ex, lse_ex = oracle.attn_fwd(qd, kd, vd, cu, scale=w.scale, causal=causal)
+    assert parity.rel_l2(o, o_ex) <= FP8_EXACT_REL_L2, name
+    assert np.abs(lse - lse_ex).max() <= parity.BF16_LSE_MAX_ABS, name
+
+
+def test_fp8_forward_large_scores_and_uneven_scales():
+    """Q and K four times larger (scores of ~±20 in log2 units: the running max moves in
+    large jumps and stays stale by up to 8) and per-head scales that differ by orders of
+    magnitude."""
+    batch, seqlen, hq, hkv = 1, 640, 4, 2
+    w, q, k, v = fp8_case("fp8-large", batch, seqlen, hq, hkv, True, 31, qk_mult=4.0)
+    q[:, 1] *= 0.01
+    k[:, 1] *= 40.0
+    q8, dq = quantize_cpu(q, hq)
+    k8, dk = quantize_cpu(k, hkv)
+    v8, dv = quantize_cpu(v, hkv)
+    o, lse = run_fwd(w, q8, k8, transpose_v_cpu(v8, batch, seqlen), dq, dk, dv)
+    qd, kd, vd = dequant(q8, dq).numpy(), dequant(k8, dk).numpy(), dequant(v8, dv).numpy()
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd, kd, vd, w.cu_seqlens().numpy(), scale=w.scale, causal=True)
+    parity.check_fwd_bf16(o, lse, o_ref, lse_ref, tag="fp8-large")
+
+
+def test_fp8_end_to_end_through_quantize():
+    """attn_fp8_quantize then attn_fwd_fp8 on the device, compared with the oracle on the
+    CPU-quantised operands (equal bytes, checked above)."""
+    batch, seqlen, hq, hkv = 2, 384, 4, 4
+    w, q, k, v = fp8_case("fp8-e2e", batch, seqlen, hq, hkv, False, 41)
+    dev = torch.device("cuda")
+    ops = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), batch)
+    o, lse = attn.attn_fwd_fp8(*ops, batch=batch, scale=w.scale, causal=False)
+    attn.attn_get_device_error()
+    q8, dq = quantize_cpu(q, hq)
+    k8, dk = quantize_cpu(k, hkv)
+    v8, dv = quantize_cpu(v, hkv)
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(dequant(q8, dq).numpy(), dequant(k8, dk).numpy(),
+                                            dequant(v8, dv).numpy(), w.cu_seqlens().numpy(), scale=w.scale)
+    parity.check_fwd_bf16(parity.to_np(o), parity.to_np(lse), o_ref, lse_ref, tag="fp8-e2e")
+
+
+def test_fp8_empty_batch_is_a_no_op():
+    dev = torch.device("cuda")
+    z8 = torch.empty(0, 2, 128, dtype=torch.uint8, device=dev)
+    vt = torch.empty(0, 128, 0, dtype=torch.uint8, device=dev)
+    ds = torch.ones(2, dtype=torch.float32, device=dev)
+    o, lse = attn.attn_fwd_fp8(z8, z8, vt, ds, ds, ds, batch=0)
+    attn.attn_get_device_error()
+    assert o.numel() == 0 and lse.numel() == 0
