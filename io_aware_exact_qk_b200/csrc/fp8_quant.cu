@@ -25,23 +25,28 @@ __device__ __forceinline__ uint8_t to_e4m3(float x) {
 }
 
 // amax over |x| per head of a [T, heads, d] bf16 tensor, as float bits (non-negative floats
-// order like their bit patterns) into amax_bits[heads] (zeroed beforehand).
-__global__ void __launch_bounds__(256) amax_per_head(const __nv_bfloat16* __restrict__ x, int64_t n, int heads, int d,
-                                                     unsigned* __restrict__ amax_bits) {
-  // one block-stride walk over 8-element groups; each group lies inside one (token, head)
-  const int64_t n8 = n / 8;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+// order like their bit patterns) into amax_bits[heads] (zeroed beforehand).  Grid
+// (token blocks, heads): d / 8 threads cover one 2d-byte row with 16-byte loads, the
+// block's rows stride over the tokens, and each warp adds its maximum with one atomic.
+__global__ void __launch_bounds__(256) amax_per_head(const __nv_bfloat16* __restrict__ x, int total_tokens,
+                                                     int heads, int d, unsigned* __restrict__ amax_bits) {
+  const int h = blockIdx.y;
+  const int gpr = d / 8;                       // 16-byte groups per row
+  const int rows = blockDim.x / gpr;           // rows per block pass
+  const int g = threadIdx.x % gpr;
+  float m = 0.f;
+  for (int t = blockIdx.x * rows + threadIdx.x / gpr; t < total_tokens; t += gridDim.x * rows) {
+    const uint4 u = *reinterpret_cast<const uint4*>(x + ((size_t)t * heads + h) * d + g * 8);
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-    float m = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __bfloat1622float2(h2[e]);
       m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
     }
-    const int head = (int)((i * 8 / d) % heads);
-    atomicMax(amax_bits + head, __float_as_uint(m));
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(amax_bits + h, __float_as_uint(m));
 }
 
 __global__ void amax_to_descale(unsigned* __restrict__ bits, int n) {
@@ -79,7 +84,7 @@ __global__ void __launch_bounds__(256) quantize_rows(const __nv_bfloat16* __rest
 __global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16* __restrict__ v, int seqlen,
                                                              int pitch, int hkv, int d, const float* __restrict__ descale,
                                                              uint8_t* __restrict__ vt8) {
-  __shared__ uint8_t tile[64][64 + 4];
+  __shared__ __align__(4) uint8_t tile[64][64 + 4];
   const int z = blockIdx.z;   // b * hkv + g
   const int g = z % hkv, b = z / hkv;
   const int c0 = blockIdx.y * 64;
@@ -93,10 +98,13 @@ __global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16
     tile[cc][tt] = to_e4m3(__fdiv_rn(x, ds));
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
-    const int cc = e / 64, tt = e % 64;
+  // four consecutive tokens per 4-byte store (pitch and t0 are multiples of 16)
+  for (int e = threadIdx.x; e < 64 * 16; e += blockDim.x) {
+    const int cc = e / 16, tt = (e % 16) * 4;
     const int t = t0 + tt;
-    if (t < pitch) vt8[((size_t)z * d + c0 + cc) * pitch + t] = tile[cc][tt];
+    if (t < pitch)
+      *reinterpret_cast<uint32_t*>(vt8 + ((size_t)z * d + c0 + cc) * pitch + t) =
+          *reinterpret_cast<const uint32_t*>(&tile[cc][tt]);
   }
 }
 
@@ -126,12 +134,14 @@ cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int
   if ((e = cudaMemsetAsync(descale_v, 0, hkv * sizeof(float), stream)) != cudaSuccess) return e;
   {
     LaunchScope scope(K_FP8_QUANTIZE, stream);
-    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), nq, hq, d,
-                                           reinterpret_cast<unsigned*>(descale_q));
-    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), nk, hkv, d,
-                                           reinterpret_cast<unsigned*>(descale_k));
-    amax_per_head<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), nk, hkv, d,
-                                           reinterpret_cast<unsigned*>(descale_v));
+    const dim3 gq(std::max(1, std::min((total_tokens + 31) / 32, grid / hq + 1)), hq);
+    const dim3 gk(std::max(1, std::min((total_tokens + 31) / 32, grid / hkv + 1)), hkv);
+    amax_per_head<<<gq, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), total_tokens, hq, d,
+                                         reinterpret_cast<unsigned*>(descale_q));
+    amax_per_head<<<gk, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), total_tokens, hkv, d,
+                                         reinterpret_cast<unsigned*>(descale_k));
+    amax_per_head<<<gk, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), total_tokens, hkv, d,
+                                         reinterpret_cast<unsigned*>(descale_v));
     amax_to_descale<<<(hq + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_q), hq);
     amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_k), hkv);
     amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_v), hkv);

@@ -54,6 +54,8 @@ constexpr float kRescaleSkip = 8.0f;       // log2 units, see file comment
 // mask selects pair c (2 of every 8 pairs, 25%, the best of 0 / 25 / 37.5 / 50% measured
 // on B200), balancing the special-function unit against the FMA pipe.
 constexpr uint32_t kEmuPairs = 0x22u;
+// The same for the FP8 forward, whose products take half the tensor-core time.
+constexpr uint32_t kEmuPairsFp8 = 0x22u;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
 constexpr int kItemSlots = 4;  // ring of work-item indices the producer hands to the other roles
@@ -474,7 +476,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           for (int c = 0; c < 64; ++c) {
             const uint64_t x = fma2(f2(s[2 * c], s[2 * c + 1]), sl2x2, negm);
             float p0, p1;
-            if ((kEmuPairs >> (c % 8)) & 1u) {
+            if (((FP8 ? kEmuPairsFp8 : kEmuPairs) >> (c % 8)) & 1u) {
               ex2_fma_pair(x, p0, p1);
             } else {
               float x0, x1;
