@@ -175,3 +175,23 @@ def test_fp8_empty_batch_is_a_no_op():
     o, lse = attn.attn_fwd_fp8(z8, z8, vt, ds, ds, ds, batch=0)
     attn.attn_get_device_error()
     assert o.numel() == 0 and lse.numel() == 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_forward_bench_size_sampled_heads(causal):
+    """The bench's FP8 configuration (B=4, H=16, N=2048, d=128) in one launch, as the bench
+    runs it; the oracle checks two whole heads of two sequences (its cost grows with N^2
+    per head, so not all 64 (sequence, head) pairs)."""
+    w = W.mha2k(causal)
+    q, k, v, _, _ = W.make_inputs(w, with_grad=False)
+    q8, dq = quantize_cpu(q, w.hq)
+    k8, dk = quantize_cpu(k, w.hkv)
+    v8, dv = quantize_cpu(v, w.hkv)
+    o, lse = run_fwd(w, q8, k8, transpose_v_cpu(v8, w.batch, w.seqlen), dq, dk, dv)
+    qd, kd, vd = dequant(q8, dq).numpy(), dequant(k8, dk).numpy(), dequant(v8, dv).numpy()
+    n = w.seqlen
+    for b, h in ((0, 3), (3, 14)):
+        rows = slice(b * n, (b + 1) * n)
+        o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd[rows, h:h + 1], kd[rows, h:h + 1], vd[rows, h:h + 1],
+                                                scale=w.scale, causal=causal)
+        parity.check_fwd_bf16(o[rows, h:h + 1], lse[h:h + 1, rows], o_ref, lse_ref, tag=f"fp8 b{b} h{h}")
