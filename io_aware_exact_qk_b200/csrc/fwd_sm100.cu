@@ -77,9 +77,9 @@ struct FwdCfg {
   static constexpr int S_KSTEPS = D * ELEM / 32;   // K steps of Q K^T
   static constexpr int PV_KSTEPS = kKeys * ELEM / 32;   // K steps of P V (8 P columns each)
   // barrier slots
-  static constexpr int B_QFULL = 0;
-  static constexpr int B_QEMPTY = 1;
-  static constexpr int B_KFULL = 2;
+  static constexpr int B_QFULL = 0;                  // 2: one per query tile
+  static constexpr int B_QEMPTY = 2;                 // 2
+  static constexpr int B_KFULL = 4;
   static constexpr int B_VFULL = B_KFULL + STAGES;
   static constexpr int B_KEMPTY = B_VFULL + STAGES;
   static constexpr int B_VEMPTY = B_KEMPTY + STAGES;
@@ -235,7 +235,8 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
   if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      uint32_t kv = 0, qi = 0;   // K/V tiles and non-empty items so far
+      uint32_t kv = 0;            // K/V tiles so far
+      uint32_t qc[2] = {0, 0};    // loads of each query tile buffer so far
       bool ok = true;
       for (int k = 0; ok; ++k) {
         // claim the next item and hand its index to the other roles
@@ -248,13 +249,21 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
         const Item it = item_from(p, idx);
         if (it.nkv == 0) continue;
         const int hk = it.h / (p.hq / p.hkv);
-        if (!mbar_wait(bar(C::B_QEMPTY), (qi & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_QFULL), ((it.n[0] > 0) + (it.n[1] > 0)) * C::TILE_BYTES);
-        for (int t = 0; t < 2; ++t)
-          if (it.n[t] > 0)
-            for (int pn = 0; pn < C::NPANEL; ++pn)
-              tma_load_3d(sQ + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, bar(C::B_QFULL), pn * C::PANEL, it.h,
-                          it.seq_start + it.q0 + t * kRows);
+        // Each query tile buffer reloads as soon as its own last QK^T of the previous item
+        // is done (under the causal mask tile 0's comes a key tile earlier), and tile 1
+        // after the item's first K tile, so the item's first product can start while the
+        // previous item's tile 1 still runs.
+        auto load_q = [&](int t) -> bool {
+          if (it.n[t] == 0) return true;
+          if (!mbar_wait(bar(C::B_QEMPTY + t), (qc[t] & 1) ^ 1, abort_flag)) return false;
+          mbar_arrive_expect_tx(bar(C::B_QFULL + t), C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_3d(sQ + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, bar(C::B_QFULL + t), pn * C::PANEL, it.h,
+                        it.seq_start + it.q0 + t * kRows);
+          ++qc[t];
+          return true;
+        };
+        if (!load_q(0)) break;
         for (int j = 0; j < it.nkv; ++j, ++kv) {
           const int s = kv % C::STAGES;
           const uint32_t ph = (kv / C::STAGES) & 1;
@@ -263,6 +272,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           for (int pn = 0; pn < C::NPANEL; ++pn)
             tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, hk,
                         it.seq_start + j * kKeys);
+          if (j == 0 && !load_q(1)) { ok = false; break; }
           if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
           if constexpr (FP8) {
@@ -275,7 +285,6 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
                           it.seq_start + j * kKeys);
           }
         }
-        ++qi;
       }
     }
   } else if (warp == 9) {
@@ -316,7 +325,8 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
             mma_ts(d_tmem, a_tmem, desc_advance(b0, kk * 16 * C::SW), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      uint32_t kv = 0, qi = 0;
+      uint32_t kv = 0;
+      uint32_t qm[2] = {0, 0};   // loads of each query tile buffer consumed
       uint32_t pc[2] = {0, 0};   // P_t tiles consumed
       uint32_t om[2] = {0, 0};   // items started per query tile (for the O-free handshake)
       bool ok = true;
@@ -325,18 +335,19 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
         if (idx < 0 || idx >= p.n_items) break;
         const Item it = item_from(p, idx);
         if (it.nkv == 0) continue;
-        int s_left = it.n[0] + it.n[1];   // QK^T MMAs still to issue; Q is free after the last
-        ok = mbar_wait(bar(C::B_QFULL), qi & 1, abort_flag);
+        int rem[2] = {it.n[0], it.n[1]};   // QK^T MMAs still to issue per tile; Q_t is free after its last
         const int s0 = kv % C::STAGES;
-        ok = ok && mbar_wait(bar(C::B_KFULL + s0), (kv / C::STAGES) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t)
+        ok = mbar_wait(bar(C::B_KFULL + s0), (kv / C::STAGES) & 1, abort_flag);
+        for (int t = 0; ok && t < 2; ++t)
           if (it.n[t] > 0) {
+            if (!mbar_wait(bar(C::B_QFULL + t), qm[t] & 1, abort_flag)) { ok = false; break; }
+            ++qm[t];
+            tc_fence_after();
             issue_qk(t, s0);
             mma_commit(bar(C::B_SFULL + t));
-            if (--s_left == 0) mma_commit(bar(C::B_QEMPTY));
+            if (--rem[t] == 0) mma_commit(bar(C::B_QEMPTY + t));
           }
+        if (!ok) break;
         mma_commit(bar(C::B_KEMPTY + s0));
         for (int j = 0; ok && j < it.nkv; ++j) {
           const uint32_t c = kv + j;
@@ -362,7 +373,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
               }
               issue_qk(t, s1);
               mma_commit(bar(C::B_SFULL + t));
-              if (--s_left == 0) mma_commit(bar(C::B_QEMPTY));
+              if (--rem[t] == 0) mma_commit(bar(C::B_QEMPTY + t));
             } else {
               mma_commit(bar(C::B_OFINAL + t));
             }
@@ -372,7 +383,6 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           if (k_next) mma_commit(bar(C::B_KEMPTY + s1));
         }
         kv += it.nkv;
-        ++qi;
       }
     }
   } else {
