@@ -106,6 +106,7 @@ struct FwdParams {
   const int32_t* cu_seqlens;
   int32_t seqlen, max_seqlen, total_tokens, hq, hkv, batch;
   int32_t n_pairs, n_items;
+  int32_t n_full;    // items [0, n_full) are two-tile items; the rest single query tiles
   float scale_log2;  // scale * log2(e), rounded to fp32
   double lse_skew;   // scale_log2 * ln 2 - scale, in double: the rounding of scale_log2
   int32_t causal;
@@ -130,7 +131,10 @@ struct Item {
 // heaviest first (the last query tiles see the most keys) within groups of
 // (head, sequence) pairs whose K / V fit in about 32 MB of L2, so that the items in flight
 // share what they stream, and lighter items fill in at the end.  Otherwise the pairs of
-// one head are consecutive (their K / V stream is shared through L2).
+// one head are consecutive (their K / V stream is shared through L2), and when the last
+// wave of two-tile items would leave more than half of the SMs idle, the pairs of that
+// wave are split into single-tile items (items n_full, n_full + 1 are the two tiles of
+// pair n_full, and so on), which fill twice as many SMs.
 __device__ __forceinline__ Item item_from(const FwdParams& p, int idx) {
   Item it;
   if (idx < 0 || idx >= p.n_items) {
@@ -139,6 +143,7 @@ __device__ __forceinline__ Item item_from(const FwdParams& p, int idx) {
     return it;
   }
   int pair;
+  int single = 0;   // 0: both tiles of the pair; 1 / 2: only its first / second tile
   if (p.causal) {
     const int pairs = p.hq * p.batch;
     const int per_grp = p.n_pairs * p.heads_per_group;
@@ -149,17 +154,22 @@ __device__ __forceinline__ Item item_from(const FwdParams& p, int idx) {
     it.h = r % p.hq;
     it.b = r / p.hq;
   } else {
-    pair = idx % p.n_pairs;
-    const int t = idx / p.n_pairs;
+    int pr = idx;
+    if (idx >= p.n_full) {
+      pr = p.n_full + (idx - p.n_full) / 2;
+      single = 1 + ((idx - p.n_full) & 1);
+    }
+    pair = pr % p.n_pairs;
+    const int t = pr / p.n_pairs;
     it.h = t % p.hq;
     it.b = t / p.hq;
   }
   it.seq_start = p.cu_seqlens ? p.cu_seqlens[it.b] : it.b * p.seqlen;
   it.len = p.cu_seqlens ? p.cu_seqlens[it.b + 1] - it.seq_start : p.seqlen;
-  it.q0 = pair * 2 * kRows;
+  it.q0 = pair * 2 * kRows + (single == 2 ? kRows : 0);
   for (int t = 0; t < 2; ++t) {
     const int r0 = it.q0 + t * kRows;
-    if (r0 >= it.len) {
+    if (r0 >= it.len || (single && t == 1)) {
       it.n[t] = 0;
     } else {
       const int kv_end = p.causal ? min(it.len, r0 + kRows) : it.len;
@@ -644,8 +654,14 @@ FwdParams fwd_params(const Problem& pb, void* o, float* lse, void* workspace) {
   p.hkv = pb.hkv;
   p.batch = pb.batch;
   p.n_pairs = (pb.max_seqlen + 2 * kRows - 1) / (2 * kRows);
-  const int64_t items = (int64_t)p.n_pairs * pb.hq * pb.batch;
+  // non-causal: split the pairs of a last wave that would fill at most half of the SMs
+  const int64_t pairs = (int64_t)p.n_pairs * pb.hq * pb.batch;
+  const int64_t ctas = sm_count_fwd();
+  const int64_t rem = pairs % ctas;
+  const int64_t split = (!pb.causal && 2 * rem <= ctas) ? rem : 0;
+  const int64_t items = pairs + split;
   p.n_items = items > INT32_MAX ? -1 : (int)items;
+  p.n_full = (int)(pairs - split);
   p.scale_log2 = pb.scale * kLog2e;
   p.lse_skew = (double)p.scale_log2 * 0.6931471805599453 - (double)pb.scale;
   p.causal = pb.causal;
