@@ -14,14 +14,20 @@ sequence (q [B n, Hq, d], k and v [B n, Hkv, d]).  Under the causal mask a chunk
 fully visible to the later chunks, causally visible to itself and hidden from the
 earlier ones.  Communication is NCCL point-to-point (over NVLink between the GPUs of one
 node); the K/V transfer of the next hop runs while the current hop is computed.
-Forward only.
+
+The backward walks the same ring.  With the full forward's O and LSE of this rank's rows
+(what ``ring_attn_fwd`` returns), the gradient over one K/V block is exactly the backward
+of the (query chunk, K/V block) pair given those O and LSE (the tutorial's 反向重算流程:
+P is recomputed from the saved LSE, D from the saved O), so dQ is the sum of the per-hop
+dQ, and each block's dK / dV accumulate as the block travels: they are passed on with it
+after every hop and arrive back at the block's owner after the last one.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
-from . import attn_fwd, attn_merge_finish, attn_merge_partial
+from . import attn_bwd, attn_fwd, attn_merge_finish, attn_merge_partial
 
 
 def ring_schedule(rank: int, world: int, causal: bool):
@@ -82,3 +88,51 @@ def ring_attn_fwd(q, k, v, batch, scale=None, causal=False, group=None, local_fw
         if s + 1 < world:
             k_cur, v_cur = k_nxt, v_nxt
     return finish(o_acc), lse_acc
+
+
+def ring_attn_bwd(q, k, v, o, do, lse, batch, scale=None, causal=False, group=None, local_bwd=None,
+                  acc_dtype=torch.float32):
+    """Gradients of the ring forward for this rank: (dq [B n, Hq, d] for its query chunk,
+    dk, dv [B n, Hkv, d] for its K/V chunk), in the dtypes of q, k, v.  ``o`` / ``lse`` are
+    this rank's rows of the full forward (``ring_attn_fwd``'s outputs), ``do`` their
+    upstream gradient.  ``local_bwd(q, k, v, causal) -> (dq, dk, dv)`` defaults to the
+    library's attn_bwd on the pair with the given o, do, lse; partial gradients are summed
+    in ``acc_dtype``."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if local_bwd is None:
+        def local_bwd(q_, k_, v_, c_):
+            return attn_bwd(q_, k_, v_, o, do, lse, scale=scale, causal=c_, batch=batch)
+    nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+    prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+    dq_acc = torch.zeros(q.shape, dtype=acc_dtype, device=q.device)
+    k_cur, v_cur = k.contiguous(), v.contiguous()
+    dk_cur = torch.zeros(k.shape, dtype=acc_dtype, device=k.device)
+    dv_cur = torch.zeros(v.shape, dtype=acc_dtype, device=v.device)
+    for s, (_, kind) in enumerate(ring_schedule(rank, world, causal)):
+        kv_reqs = []
+        if s + 1 < world:
+            # the next hop's block moves while this hop is computed
+            k_nxt, v_nxt = torch.empty_like(k_cur), torch.empty_like(v_cur)
+            kv_reqs = dist.batch_isend_irecv([
+                dist.P2POp(dist.isend, k_cur, nxt, group), dist.P2POp(dist.irecv, k_nxt, prv, group),
+                dist.P2POp(dist.isend, v_cur, nxt, group), dist.P2POp(dist.irecv, v_nxt, prv, group)])
+        if kind is not None:
+            dq_p, dk_p, dv_p = local_bwd(q, k_cur, v_cur, kind == "causal")
+            dq_acc += dq_p.to(acc_dtype)
+            dk_cur += dk_p.to(acc_dtype)
+            dv_cur += dv_p.to(acc_dtype)
+        # the block's gradients so far go on with it (after the last hop: to its owner)
+        g_reqs = []
+        if world > 1:
+            dk_in, dv_in = torch.empty_like(dk_cur), torch.empty_like(dv_cur)
+            g_reqs = dist.batch_isend_irecv([
+                dist.P2POp(dist.isend, dk_cur, nxt, group), dist.P2POp(dist.irecv, dk_in, prv, group),
+                dist.P2POp(dist.isend, dv_cur, nxt, group), dist.P2POp(dist.irecv, dv_in, prv, group)])
+        for r in kv_reqs + g_reqs:
+            r.wait()
+        if world > 1:
+            dk_cur, dv_cur = dk_in, dv_in
+        if s + 1 < world:
+            k_cur, v_cur = k_nxt, v_nxt
+    return dq_acc.to(q.dtype), dk_cur.to(k.dtype), dv_cur.to(v.dtype)

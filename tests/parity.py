@@ -142,9 +142,11 @@ def check_sampled(w, inputs, outputs, picks, seed=0, tag="", given=False, fp32_l
     (sequence, GQA group) slice -- every row enters the statistics -- and the comparison
     covers O/LSE and dQ on sampled query rows and dK/dV on sampled keys.
 
-    given=True compares the backward as a function of its inputs: the oracle's backward
-    takes the GPU forward's O (for D) and LSE (for P), as attn_bwd does; otherwise the
-    reference is the exact gradient.  fp32_lse_bound_rows=True checks LSE against
+    given=True compares the backward as a function of its inputs: the oracle's own forward
+    of the slice, stored as attn_fwd stores it (O rounded to bf16, LSE to fp32), is
+    written over the slice of the device O / LSE, the GPU backward runs again on them,
+    and the oracle's backward takes the same stored O (for D) and LSE (for P); no value
+    the GPU computed enters the oracle.  Otherwise the reference is the exact gradient.  fp32_lse_bound_rows=True checks LSE against
     max(1e-3, fp32_lse_bound) per row instead of 1e-3 (for scores far above fp32's
     exact-integer range, where 1e-3 is below a few ulps of the LSE itself)."""
     q, k, v, do, cu = inputs
@@ -164,11 +166,22 @@ def check_sampled(w, inputs, outputs, picks, seed=0, tag="", given=False, fp32_l
         keys = sample_indices(n, rng)
         o_full = to_np(o[t0:t1, hs])
         lse_full = to_np(lse[hs, t0:t1])
-        extra = dict(o=o_full, lse=lse_full) if given else {}
+        grads = (dq, dk, dv)
+        extra = {}
+        if given:
+            o_or, lse_or = oracle.attn_fwd(q[sl], k[ks], v[ks], scale=w.scale, causal=w.causal)
+            o_st = torch.from_numpy(o_or).to(torch.bfloat16)
+            lse_st = torch.from_numpy(lse_or).to(torch.float32)
+            o_dev, lse_dev = o.clone(), lse.clone()
+            o_dev[t0:t1, hs] = o_st.to(o_dev.device)
+            lse_dev[hs, t0:t1] = lse_st.to(lse_dev.device)
+            grads = gpu_bwd(w, q, k, v, o_dev, do, lse_dev, cu)
+            del o_dev, lse_dev
+            extra = dict(o=o_st.double().numpy(), lse=lse_st.double().numpy())
         dq_r, dk_r, dv_r, o_r, lse_r = oracle.attn_bwd(q[sl], k[ks], v[ks], do[sl], scale=w.scale, causal=w.causal,
                                                        rows=rows, keys=keys, **extra)
         if given:   # the forward reference is the oracle's own forward either way
-            o_r, lse_r = oracle.attn_fwd(q[sl], k[ks], v[ks], scale=w.scale, causal=w.causal, rows=rows)
+            o_r, lse_r = o_or, lse_or
         tg = f"{tag} seq{b} g{g}"
         lse_tol = None
         if fp32_lse_bound_rows:
@@ -176,7 +189,8 @@ def check_sampled(w, inputs, outputs, picks, seed=0, tag="", given=False, fp32_l
             lse_tol = np.stack([fp32_lse_bound(to_np(q[t0:t1, h])[rows], k_np, w.scale, w.causal, rows)
                                 for h in range(g * G, (g + 1) * G)])
         check_fwd_bf16(o_full[rows], lse_full[:, rows], o_r[rows], lse_r[:, rows], tag=tg, lse_tol=lse_tol)
-        errs = check_grads_bf16((dq[t0:t1, hs], dk[t0:t1, g:g + 1], dv[t0:t1, g:g + 1]),
+        gq, gk, gv = grads
+        errs = check_grads_bf16((gq[t0:t1, hs], gk[t0:t1, g:g + 1], gv[t0:t1, g:g + 1]),
                                 (dq_r, dk_r, dv_r), rows=rows, keys=keys, tag=tg)
         report.append((b, g, errs))
     return report

@@ -63,7 +63,9 @@ def test_gqa8k_stability_x30():
       - gradients: with P nearly one-hot, dS = P (dP - D) is a cancellation that
         amplifies the rounding of the saved bf16 O (through D) about a hundredfold
         relative to dS, so the backward is compared as a function of its inputs -- the
-        oracle's backward takes the same saved O and LSE -- at the usual 1e-2."""
+        oracle's forward of each sampled slice, stored as bf16 O and fp32 LSE, is given
+        to both the GPU backward (rerun on it) and the oracle's backward -- at the usual
+        1e-2."""
     w = W.gqa8k(stability=True)
     _run_and_check(w, _inputs("gqa8k_x30"), [(0, 0), (1, 7)], seed=8, given=True, fp32_lse_bound_rows=True)
 

@@ -1,10 +1,13 @@
-"""Ring attention's GPU arithmetic: the forward on chunk pairs and the merge kernels.
+"""Ring attention's GPU arithmetic: the forward and backward on chunk pairs and the merge
+kernels.
 
 This run has one GPU, so the ranks of the ring are emulated in turn in one process: for
 every rank the hops of ``ring_schedule`` are executed with the library's kernels
 (attn_fwd on the (query chunk, K/V chunk) pair, attn_merge_partial, attn_merge_finish),
 and the rows of all ranks together must match the fp64 oracle over the whole sequences
-with the forward's tolerances.  The point-to-point passing of the blocks between real
+with the forward's tolerances; the backward's per-hop gradients, summed the way the
+travelling dK / dV are, must match the oracle's gradient at the backward's tolerance.
+The point-to-point passing of the blocks between real
 ranks is covered by the gloo test on the CPU; the driver itself runs here as a one-rank
 NCCL group.
 """
@@ -19,7 +22,7 @@ import torch.distributed as dist
 import attn_workloads as W
 import io_aware_exact_qk_b200 as attn
 import oracle
-from io_aware_exact_qk_b200.ring import ring_attn_fwd, ring_schedule
+from io_aware_exact_qk_b200.ring import ring_attn_bwd, ring_attn_fwd, ring_schedule
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -63,6 +66,45 @@ def test_emulated_ring_matches_full_attention(world, causal, d):
                               o_ref[:, mine], lse_ref[:, :, mine], tag=f"rank {r}")
 
 
+@pytest.mark.parametrize("world,causal,d", [(2, True, 128), (3, False, 64), (4, True, 32)])
+def test_emulated_ring_backward_matches_the_gradient(world, causal, d):
+    """Every rank's hops run attn_bwd on its (query chunk, K/V block) pairs with its rows of
+    the full forward's O and LSE; dQ sums over the rank's hops, dK / dV of a block over the
+    ranks it visits.  The stored O (bf16) and LSE (fp32) are the oracle's forward, given to
+    the oracle's backward as well (the backward as a function of its inputs)."""
+    batch, n, hq, hkv = 2, 256 if d == 128 else 200, 8, 2
+    N = world * n
+    w = W.custom("ring-bwd", [N] * batch, hq, hkv, d, causal, 3300 + world)
+    q, k, v, do, cu = W.make_inputs(w)
+    o_or, lse_or = oracle.attn_fwd(q, k, v, cu.numpy(), scale=w.scale, causal=causal)
+    o_st = torch.from_numpy(o_or).to(torch.bfloat16)
+    lse_st = torch.from_numpy(lse_or).to(torch.float32)
+    qs, ks, vs, dos, os_ = (_chunks(t, batch, N, world) for t in (q, k, v, do, o_st))
+    lse_b = lse_st.reshape(hq, batch, N)
+    lses = [lse_b[:, :, r * n:(r + 1) * n].reshape(hq, batch * n).contiguous().cuda() for r in range(world)]
+    dq = [torch.zeros(batch * n, hq, d, device="cuda") for _ in range(world)]
+    dk = [torch.zeros(batch * n, hkv, d, device="cuda") for _ in range(world)]
+    dv = [torch.zeros(batch * n, hkv, d, device="cuda") for _ in range(world)]
+    for r in range(world):
+        for j, kind in ring_schedule(r, world, causal):
+            if kind is None:
+                continue
+            gq, gk, gv = attn.attn_bwd(qs[r], ks[j], vs[j], os_[r], dos[r], lses[r], scale=w.scale,
+                                       causal=kind == "causal", batch=batch)
+            dq[r] += gq.float()
+            dk[j] += gk.float()
+            dv[j] += gv.float()
+    attn.attn_get_device_error()
+    dq_r, dk_r, dv_r, _, _ = oracle.attn_bwd(q, k, v, do, cu.numpy(), scale=w.scale, causal=causal,
+                                             o=o_st.double().numpy(), lse=lse_st.double().numpy())
+
+    def whole(parts, h):
+        return torch.stack([p.cpu().reshape(batch, n, h, d) for p in parts], dim=1).reshape(batch * N, h, d)
+
+    parity.check_grads_bf16((whole(dq, hq), whole(dk, hkv), whole(dv, hkv)), (dq_r, dk_r, dv_r),
+                            tag=f"ring bwd W={world}")
+
+
 def test_merge_kernel_edge_cases():
     T, hq, d = 37, 4, 128
     g = torch.Generator().manual_seed(5)
@@ -101,5 +143,15 @@ def test_driver_as_a_one_rank_nccl_group():
         attn.attn_get_device_error()
         o_ref, lse_ref = oracle.attn_fwd(q, k, v, cu.numpy(), scale=w.scale, causal=True)
         parity.check_fwd_bf16(o, lse, o_ref, lse_ref, tag="one-rank ring")
+        # the backward driver on the oracle's stored forward
+        do = W.make_inputs(W.custom("ring-do", [N] * batch, hq, hkv, d, True, 3201))[3]
+        o_st = torch.from_numpy(o_ref).to(torch.bfloat16)
+        lse_st = torch.from_numpy(lse_ref).to(torch.float32)
+        dq, dk, dv = ring_attn_bwd(q.cuda(), k.cuda(), v.cuda(), o_st.cuda(), do.cuda(), lse_st.cuda(), batch,
+                                   scale=w.scale, causal=True)
+        attn.attn_get_device_error()
+        dq_r, dk_r, dv_r, _, _ = oracle.attn_bwd(q, k, v, do, cu.numpy(), scale=w.scale, causal=True,
+                                                 o=o_st.double().numpy(), lse=lse_st.double().numpy())
+        parity.check_grads_bf16((dq, dk, dv), (dq_r, dk_r, dv_r), tag="one-rank ring bwd")
     finally:
         dist.destroy_process_group()

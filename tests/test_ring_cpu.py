@@ -1,10 +1,11 @@
-"""The ring-attention driver over a real multi-process group (gloo on CPU).
+"""The ring-attention drivers over a real multi-process group (gloo on CPU).
 
-Each rank holds one chunk of every sequence and runs ``ring_attn_fwd``, the same driver
-the GPUs run, with its two compute steps swapped for CPU stand-ins (the local attention
-from the fp64 oracle, the merge in float64 numpy) -- the schedule, the masks of every hop
-and the point-to-point passing of the K/V blocks are what is under test here.  The rows
-gathered from all ranks must equal the oracle's forward over the whole sequences.
+Each rank holds one chunk of every sequence and runs ``ring_attn_fwd`` and
+``ring_attn_bwd``, the same drivers the GPUs run, with their compute steps swapped for
+CPU stand-ins (the local attention and its backward from the fp64 oracle, the merge in
+float64) -- the schedule, the masks of every hop, the point-to-point passing of the K/V
+blocks and of their travelling dK / dV are what is under test here.  The rows gathered
+from all ranks must equal the oracle's forward and gradient over the whole sequences.
 """
 import socket
 
@@ -49,29 +50,46 @@ def _merge64(o_acc, lse_acc, o_p, lse_p, first):
     lse_acc.copy_(m + torch.log(s))
 
 
+def _local_oracle_bwd(batch, scale, o, do, lse):
+    def f(q, k, v, causal):
+        n = q.shape[0] // batch
+        cu = np.arange(batch + 1, dtype=np.int32) * n
+        dq, dk, dv, _, _ = oracle.attn_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), cu, scale=scale,
+                                           causal=causal, threads=1, o=o.numpy(), lse=lse.numpy())
+        return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+    return f
+
+
+def _full_inputs(batch, N, hq, hkv, d):
+    g = torch.Generator().manual_seed(77)
+    q = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
+    k = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+    v = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+    do = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
+    return q, k, v, do
+
+
 def _worker(rank, world, port, batch, n, hq, hkv, d, causal, out):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
-        from io_aware_exact_qk_b200.ring import ring_attn_fwd
-        g = torch.Generator().manual_seed(77)
-        N = world * n
-        q = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
-        k = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
-        v = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+        from io_aware_exact_qk_b200.ring import ring_attn_bwd, ring_attn_fwd
+        q, k, v, do = _full_inputs(batch, world * n, hq, hkv, d)
         mine = slice(rank * n, (rank + 1) * n)
-        qc, kc, vc = (t[:, mine].reshape(batch * n, t.shape[2], d).contiguous() for t in (q, k, v))
+        qc, kc, vc, doc = (t[:, mine].reshape(batch * n, t.shape[2], d).contiguous() for t in (q, k, v, do))
         scale = 1.0 / np.sqrt(d)
         o, lse = ring_attn_fwd(qc, kc, vc, batch, scale=scale, causal=causal, local_fwd=_local_oracle(batch, scale),
                                merge=_merge64, finish=lambda oa: oa, acc_dtype=torch.float64)
-        out[rank] = (o.numpy(), lse.numpy())
+        dq, dk, dv = ring_attn_bwd(qc, kc, vc, o, doc, lse, batch, scale=scale, causal=causal,
+                                   local_bwd=_local_oracle_bwd(batch, scale, o, doc, lse), acc_dtype=torch.float64)
+        out[rank] = (o.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy())
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [1, 2, 3])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ring_forward_equals_full_attention(world, causal):
+def test_ring_forward_and_backward_equal_full_attention(world, causal):
     batch, n, hq, hkv, d = 2, 5, 4, 2, 8
     port = _free_port()
     ctx = mp.get_context("spawn")
@@ -85,21 +103,23 @@ def test_ring_forward_equals_full_attention(world, causal):
             p.join(timeout=120)
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
         res = dict(out)
-    g = torch.Generator().manual_seed(77)
     N = world * n
-    q = torch.randn(batch, N, hq, d, generator=g, dtype=torch.float64)
-    k = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
-    v = torch.randn(batch, N, hkv, d, generator=g, dtype=torch.float64)
+    q, k, v, do = _full_inputs(batch, N, hq, hkv, d)
     cu = np.arange(batch + 1, dtype=np.int32) * N
-    o_ref, lse_ref = oracle.attn_fwd(q.reshape(-1, hq, d).numpy(), k.reshape(-1, hkv, d).numpy(),
-                                     v.reshape(-1, hkv, d).numpy(), cu, causal=causal)
-    o_ref = o_ref.reshape(batch, N, hq, d)
+    dq_ref, dk_ref, dv_ref, o_ref, lse_ref = oracle.attn_bwd(
+        q.reshape(-1, hq, d).numpy(), k.reshape(-1, hkv, d).numpy(), v.reshape(-1, hkv, d).numpy(),
+        do.reshape(-1, hq, d).numpy(), cu, causal=causal)
+    o_ref, dq_ref = o_ref.reshape(batch, N, hq, d), dq_ref.reshape(batch, N, hq, d)
+    dk_ref, dv_ref = dk_ref.reshape(batch, N, hkv, d), dv_ref.reshape(batch, N, hkv, d)
     lse_ref = lse_ref.reshape(hq, batch, N)
     for r in range(world):
-        o, lse = res[r]
+        o, lse, dq, dk, dv = res[r]
         mine = slice(r * n, (r + 1) * n)
         np.testing.assert_allclose(o.reshape(batch, n, hq, d), o_ref[:, mine], rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse.reshape(hq, batch, n), lse_ref[:, :, mine], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dq.reshape(batch, n, hq, d), dq_ref[:, mine], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(dk.reshape(batch, n, hkv, d), dk_ref[:, mine], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(dv.reshape(batch, n, hkv, d), dv_ref[:, mine], rtol=0, atol=1e-10)
 
 
 def test_ring_schedule_visits_every_block_once():
