@@ -183,17 +183,17 @@ attn_status attn_merge_finish(const float *o_acc, void *o, int32_t total_tokens,
 /* FP8 (e4m3) forward operands.  The "Flash-Attention" concept page names FP8 attention
  * (FlashAttention-3 on H100, 观察 2) and quantised attention with scaling (设计空间, 路线 4);
  * the scaling chosen here is one factor per head and tensor.
- * Reads bf16 q [batch*seqlen, hq, 128], k and v [batch*seqlen, hkv, 128] (a fixed-length
- * batch; d must be 128) and writes, all on the device, caller-allocated, 16-byte aligned:
+ * Reads bf16 q [batch*seqlen, hq, d], k and v [batch*seqlen, hkv, d] (a fixed-length
+ * batch; d = 64 or 128) and writes, all on the device, caller-allocated, 16-byte aligned:
  *   descale_q [hq], descale_k [hkv], descale_v [hkv] float32: amax over the head / 448
  *       (1 for an all-zero head), 448 being the largest finite e4m3 value;
- *   q8 [batch*seqlen, hq, 128], k8 [batch*seqlen, hkv, 128] bytes: e4m3 of x / descale
+ *   q8 [batch*seqlen, hq, d], k8 [batch*seqlen, hkv, d] bytes: e4m3 of x / descale
  *       (fp32 division, round to nearest even, saturating);
- *   vt8 [batch*hkv][128][pitch] bytes, pitch = seqlen rounded up to a multiple of 16:
+ *   vt8 [batch*hkv][d][pitch] bytes, pitch = seqlen rounded up to a multiple of 16:
  *       the same for v, transposed per (sequence, kv head) so that tokens are contiguous;
  *       the padding columns are zero.
- * Errors: ATTN_ERR_UNSUPPORTED for d != 128; ATTN_ERR_INVALID_ARG for NULL or unaligned
- * pointers and negative sizes.  Asynchronous on `stream`. */
+ * Errors: ATTN_ERR_UNSUPPORTED for d other than 64 or 128; ATTN_ERR_INVALID_ARG for NULL
+ * or unaligned pointers and negative sizes.  Asynchronous on `stream`. */
 attn_status attn_fp8_quantize(const void *q, const void *k, const void *v,
                               int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d,
                               void *q8, void *k8, void *vt8,
@@ -202,13 +202,14 @@ attn_status attn_fp8_quantize(const void *q, const void *k, const void *v,
 /* FP8 forward: O = softmax(scale * (dq Q8)(dk K8)^T [+ causal mask]) (dv V8), per head
  * (the tutorial's 标准注意力三步 on the dequantised operands, reached by the same online
  * softmax as attn_fwd, with both products on e4m3 tensor cores).  Inputs are what
- * attn_fp8_quantize writes (same layouts, same fixed-length batch, d = 128).  The
+ * attn_fp8_quantize writes (same layouts, same fixed-length batch, d = 64 or 128).  The
  * probabilities that multiply V are rounded to e4m3 without a scale: the running row
  * maximum only moves when a tile's maximum exceeds it by more than 8 (log2 units), so every
  * probability lies in [0, 256], inside e4m3's range.  The row sums use the unrounded
- * probabilities.  Writes o [batch*seqlen, hq, 128] bf16 and lse [hq, batch*seqlen] float32
+ * probabilities.  Writes o [batch*seqlen, hq, d] bf16 and lse [hq, batch*seqlen] float32
  * (of the dequantised scores).  Workspace: attn_fwd_workspace_size(..., ATTN_BF16) = 256
- * bytes, as for attn_fwd.  Errors as attn_fwd; d != 128 is ATTN_ERR_UNSUPPORTED. */
+ * bytes, as for attn_fwd.  Errors as attn_fwd; d other than 64 or 128 is
+ * ATTN_ERR_UNSUPPORTED. */
 attn_status attn_fwd_fp8(const void *q8, const void *k8, const void *vt8,
                          const float *descale_q, const float *descale_k, const float *descale_v,
                          int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d,

@@ -194,7 +194,9 @@ bool encode_tma_u8_3d(void* tmap_out, const void* base, int dim0, int dim1, int 
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(reinterpret_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   box0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   box0 == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                   : box0 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -221,7 +223,7 @@ namespace {
 // Shapes of the FP8 calls: a fixed-length batch (batch sequences of seqlen tokens), d = 128.
 attn_status check_fp8(int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
                       Problem* pb) {
-  if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 forward needs head dim 128 (got %d)", d);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 forward needs head dim 64 or 128 (got %d)", d);
   if (batch < 0 || seqlen < 0) return fail(ATTN_ERR_INVALID_ARG, "negative batch / seqlen");
   if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
   if ((int64_t)batch * hkv > 65535) return fail(ATTN_ERR_UNSUPPORTED, "batch * hkv must be <= 65535");

@@ -61,11 +61,13 @@ constexpr int kThreads = 320;
 constexpr int kItemSlots = 4;  // ring of work-item indices the producer hands to the other roles
 
 // FP8: Q, K and V^T (per-head transposed V) are e4m3 tiles and both products run as
-// kind::f8f6f4 with 32-element K steps; P goes to TMEM as four e4m3 per column.
+// kind::f8f6f4 with 32-element K steps; P goes to TMEM as four e4m3 per column.  A Q / K
+// row is d bytes (128: one 128-byte swizzle span; 64: the 64-byte swizzle), a V^T row is
+// 128 keys = 128 bytes whatever d is.
 template <int D, bool FP8 = false>
 struct FwdCfg {
   static constexpr int ELEM = FP8 ? 1 : 2;         // bytes per Q/K/V element
-  static constexpr int SW = (FP8 || D >= 64) ? 128 : 64;   // swizzle span == SMEM row pitch (bytes)
+  static constexpr int SW = D * ELEM >= 128 ? 128 : 64;   // swizzle span == SMEM row pitch (bytes)
   static constexpr int PANEL = SW / ELEM;          // elements per panel row
   static constexpr int NPANEL = D / PANEL;         // panels per tile
   static constexpr int PANEL_BYTES = kRows * SW;   // one panel of a 128-row tile
@@ -73,6 +75,9 @@ struct FwdCfg {
   static constexpr int STAGES = FP8 ? 4 : (D == 128 ? 2 : (D == 64 ? 3 : 4));
   static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;   // descriptor swizzle code
   static constexpr int SBO = 8 * SW;               // bytes between 8-row swizzle atoms
+  // FP8 V^T tile: d rows of 128 keys, always the 128-byte swizzle
+  static constexpr uint32_t VT_SWZ = 2u;
+  static constexpr int VT_SBO = 1024;
   static constexpr int KSTEPS_PER_PANEL = SW / 32; // 32-byte K steps inside one panel
   static constexpr int S_KSTEPS = D * ELEM / 32;   // K steps of Q K^T
   static constexpr int PV_KSTEPS = kKeys * ELEM / 32;   // K steps of P V (8 P columns each)
@@ -309,7 +314,8 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
       // instructions -- this single thread's issue rate bounds the tensor core.
       const uint64_t q_desc = smem_desc(sQ, 16, C::SBO, C::SWZ);
       const uint64_t k_desc = smem_desc(sK, 16, C::SBO, C::SWZ);
-      const uint64_t v_desc = FP8 ? smem_desc(sV, 16, C::SBO, C::SWZ) : smem_desc(sV, C::PANEL_BYTES, C::SBO, C::SWZ);
+      const uint64_t v_desc = FP8 ? smem_desc(sV, 16, C::VT_SBO, C::VT_SWZ)
+                                  : smem_desc(sV, C::PANEL_BYTES, C::SBO, C::SWZ);
       auto issue_qk = [&](int t, int s) {
         const uint32_t d_tmem = tmem + t * kKeys;
         const uint64_t a0 = desc_advance(q_desc, (uint32_t)t * C::TILE_BYTES);
@@ -716,18 +722,18 @@ cudaError_t launch_fwd_bf16(const Problem& pb, const void* q, const void* k, con
   }
 }
 
-cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, const void* vt8,
-                           const float* descale_q, const float* descale_k, const float* descale_v, void* o,
-                           float* lse, void* workspace, cudaStream_t stream) {
-  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
-  if (pb.d != 128 || pb.cu_seqlens != nullptr) return cudaErrorInvalidValue;
-  constexpr int D = 128;
+namespace {
+
+template <int D>
+cudaError_t launch_fwd_fp8_d(const Problem& pb, const void* q8, const void* k8, const void* vt8,
+                             const float* descale_q, const float* descale_k, const float* descale_v, void* o,
+                             float* lse, void* workspace, cudaStream_t stream) {
   const int sp = fp8_vt_pitch(pb.seqlen);
   alignas(64) CUtensorMap tq, tk, tv;
-  // Q8, K8: [tokens, heads, 128] bytes, one 128-byte swizzled row per token
+  // Q8, K8: [tokens, heads, d] bytes, one d-byte swizzled row per token
   if (!encode_tma_u8_3d(&tq, q8, D, pb.hq, pb.total_tokens, (uint64_t)D, (uint64_t)pb.hq * D, D, 1, kRows) ||
       !encode_tma_u8_3d(&tk, k8, D, pb.hkv, pb.total_tokens, (uint64_t)D, (uint64_t)pb.hkv * D, D, 1, kKeys) ||
-      // V^T: [batch * hkv][128][sp] bytes, boxes of 128 keys x 128 features
+      // V^T: [batch * hkv][d][sp] bytes, boxes of 128 keys x d features
       !encode_tma_u8_3d(&tv, vt8, sp, D, pb.batch * pb.hkv, (uint64_t)sp, (uint64_t)D * sp, kKeys, D, 1))
     return cudaErrorInvalidValue;
   FwdParams p = fwd_params<D, true>(pb, o, lse, workspace);
@@ -735,6 +741,23 @@ cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, co
   p.descale_k = descale_k;
   p.descale_v = descale_v;
   return launch_fwd_common<D, true>(fwd_fp8_sm100<D>, K_FWD_FP8, tq, tk, tv, p, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, const void* vt8,
+                           const float* descale_q, const float* descale_k, const float* descale_v, void* o,
+                           float* lse, void* workspace, cudaStream_t stream) {
+  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
+  if (pb.cu_seqlens != nullptr) return cudaErrorInvalidValue;
+  switch (pb.d) {
+    case 64:
+      return launch_fwd_fp8_d<64>(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace, stream);
+    case 128:
+      return launch_fwd_fp8_d<128>(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace attn

@@ -57,8 +57,8 @@ cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_par
                                  int total_tokens, int hq, int d, int first, cudaStream_t stream);
 cudaError_t launch_merge_finish(const float* o_acc, void* o, int total_tokens, int hq, int d, cudaStream_t stream);
 
-// FP8 forward (d = 128, fixed-length batches): e4m3 Q8, K8 [tokens, heads, 128] and V^T
-// [batch * hkv][128][fp8_vt_pitch(seqlen)] with per-head descales; bf16 O, fp32 LSE.
+// FP8 forward (d = 64 or 128, fixed-length batches): e4m3 Q8, K8 [tokens, heads, d] and
+// V^T [batch * hkv][d][fp8_vt_pitch(seqlen)] with per-head descales; bf16 O, fp32 LSE.
 inline int fp8_vt_pitch(int seqlen) { return (seqlen + 15) / 16 * 16; }
 cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, const void* vt8,
                            const float* descale_q, const float* descale_k, const float* descale_v, void* o,
@@ -116,8 +116,8 @@ bool encode_tma_3d(void* tmap_out, const void* base, int d, int heads, int rows,
 bool encode_tma_3d_box(void* tmap_out, const void* base, int d, int heads, int rows, int box_inner, int box_heads,
                        int box_rows);
 // A 3-D tensor of bytes (e4m3) with extents dim0 (contiguous) x dim1 x dim2, the byte
-// strides of dims 1 and 2, and a box0 x box1 x box2 box; a 128-byte box row uses the
-// 128-byte swizzle.
+// strides of dims 1 and 2, and a box0 x box1 x box2 box; a 128- or 64-byte box row uses
+// the swizzle of that span.
 bool encode_tma_u8_3d(void* tmap_out, const void* base, int dim0, int dim1, int dim2, uint64_t stride1,
                       uint64_t stride2, int box0, int box1, int box2);
 // The same over an fp32 [rows, heads, d] tensor; a 32-float (128-byte) box row uses the

@@ -144,7 +144,7 @@ def _fwd_fp8(lib, d=128, batch=1, seqlen=64, hq=2, hkv=2, ptr=0x1000, o=0x1000, 
 
 
 def test_fp8_calls_reject_bad_arguments_on_host(lib):
-    assert _fwd_fp8(lib, d=64) == attn.ATTN_ERR_UNSUPPORTED            # e4m3 path is d = 128 only
+    assert _fwd_fp8(lib, d=32) == attn.ATTN_ERR_UNSUPPORTED            # e4m3 path is d = 64 or 128
     assert _fwd_fp8(lib, ptr=None) == attn.ATTN_ERR_INVALID_ARG
     assert _fwd_fp8(lib, o=0x1008) == attn.ATTN_ERR_INVALID_ARG         # misaligned output
     assert _fwd_fp8(lib, wsb=0) == attn.ATTN_ERR_INVALID_ARG            # needs the 256-byte counter

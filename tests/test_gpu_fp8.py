@@ -58,20 +58,25 @@ def dequant(x8, ds):
     return x8.view(torch.float8_e4m3fn).double() * ds.double()[None, :, None]
 
 
-def fp8_case(name, batch, seqlen, hq, hkv, causal, seed, qk_mult=1.0):
-    w = W.custom(name, [seqlen] * batch, hq, hkv, 128, causal, seed, qk_mult=qk_mult)
+def fp8_case(name, batch, seqlen, hq, hkv, causal, seed, qk_mult=1.0, d=128):
+    w = W.custom(name, [seqlen] * batch, hq, hkv, d, causal, seed, qk_mult=qk_mult)
     q, k, v, _, _ = W.make_inputs(w, with_grad=False)
     return w, q, k, v
 
 
 CASES = [
-    # name, batch, seqlen, hq, hkv, causal, seed
-    ("fp8-1000-gqa", 2, 1000, 4, 2, False, 11),
-    ("fp8-1000-gqa-causal", 2, 1000, 4, 2, True, 12),
-    ("fp8-257", 1, 257, 2, 2, False, 13),
-    ("fp8-257-causal", 1, 257, 2, 1, True, 14),
-    ("fp8-2048-causal", 1, 2048, 2, 2, True, 15),
-    ("fp8-77", 3, 77, 2, 1, False, 16),
+    # name, batch, seqlen, hq, hkv, causal, seed, d
+    ("fp8-1000-gqa", 2, 1000, 4, 2, False, 11, 128),
+    ("fp8-1000-gqa-causal", 2, 1000, 4, 2, True, 12, 128),
+    ("fp8-257", 1, 257, 2, 2, False, 13, 128),
+    ("fp8-257-causal", 1, 257, 2, 1, True, 14, 128),
+    ("fp8-2048-causal", 1, 2048, 2, 2, True, 15, 128),
+    ("fp8-77", 3, 77, 2, 1, False, 16, 128),
+    ("fp8-1", 2, 1, 2, 2, True, 20, 128),
+    ("fp8-d64-1000-gqa", 2, 1000, 4, 2, False, 17, 64),
+    ("fp8-d64-300-causal", 1, 300, 8, 2, True, 18, 64),
+    ("fp8-d64-2048-causal", 1, 2048, 2, 2, True, 19, 64),
+    ("fp8-d64-33", 3, 33, 2, 1, False, 21, 64),
 ]
 
 
@@ -85,8 +90,8 @@ def run_fwd(w, q8, k8, vt8, dq, dk, dv):
 
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_fp8_quantize_bit_exact(case):
-    name, batch, seqlen, hq, hkv, causal, seed = case
-    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed)
+    name, batch, seqlen, hq, hkv, causal, seed, d = case
+    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed, d=d)
     dev = torch.device("cuda")
     q8, k8, vt8, dq, dk, dv = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), batch)
     attn.attn_get_device_error()
@@ -96,7 +101,7 @@ def test_fp8_quantize_bit_exact(case):
     assert torch.equal(dq.cpu(), dq_ref) and torch.equal(dk.cpu(), dk_ref) and torch.equal(dv.cpu(), dv_ref)
     assert torch.equal(q8.cpu(), q8_ref)
     assert torch.equal(k8.cpu(), k8_ref)
-    assert tuple(vt8.shape) == (batch * hkv, 128, pitch_of(seqlen))
+    assert tuple(vt8.shape) == (batch * hkv, d, pitch_of(seqlen))
     assert torch.equal(vt8.cpu(), transpose_v_cpu(v8_ref, batch, seqlen))
 
 
@@ -116,8 +121,8 @@ def test_fp8_quantize_zero_head_and_outlier_head():
 
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_fp8_forward_matches_oracle(case):
-    name, batch, seqlen, hq, hkv, causal, seed = case
-    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed)
+    name, batch, seqlen, hq, hkv, causal, seed, d = case
+    w, q, k, v = fp8_case(name, batch, seqlen, hq, hkv, causal, seed, d=d)
     q8, dq = quantize_cpu(q, hq)
     k8, dk = quantize_cpu(k, hkv)
     v8, dv = quantize_cpu(v, hkv)
