@@ -132,27 +132,30 @@ cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int
   if ((e = cudaMemsetAsync(descale_q, 0, hq * sizeof(float), stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(descale_k, 0, hkv * sizeof(float), stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(descale_v, 0, hkv * sizeof(float), stream)) != cudaSuccess) return e;
-  {
+  // every launch is counted (and, while timing is on, timed) as one fp8_quantize kernel
+  auto launch = [&](auto kernel, dim3 g, auto... args) {
     LaunchScope scope(K_FP8_QUANTIZE, stream);
-    const dim3 gq(std::max(1, std::min((total_tokens + 31) / 32, grid / hq + 1)), hq);
-    const dim3 gk(std::max(1, std::min((total_tokens + 31) / 32, grid / hkv + 1)), hkv);
-    amax_per_head<<<gq, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), total_tokens, hq, d,
-                                         reinterpret_cast<unsigned*>(descale_q));
-    amax_per_head<<<gk, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), total_tokens, hkv, d,
-                                         reinterpret_cast<unsigned*>(descale_k));
-    amax_per_head<<<gk, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), total_tokens, hkv, d,
-                                         reinterpret_cast<unsigned*>(descale_v));
-    amax_to_descale<<<(hq + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_q), hq);
-    amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_k), hkv);
-    amax_to_descale<<<(hkv + 255) / 256, 256, 0, stream>>>(reinterpret_cast<unsigned*>(descale_v), hkv);
-    quantize_rows<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), nq, hq, d, descale_q,
-                                           static_cast<uint8_t*>(q8));
-    quantize_rows<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), nk, hkv, d, descale_k,
-                                           static_cast<uint8_t*>(k8));
-    quantize_v_transposed<<<dim3((pitch + 63) / 64, d / 64, batch * hkv), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(v), seqlen, pitch, hkv, d, descale_v, static_cast<uint8_t*>(vt8));
-    e = cudaGetLastError();
-  }
+    kernel<<<g, 256, 0, stream>>>(args...);
+  };
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  auto* bq = reinterpret_cast<unsigned*>(descale_q);
+  auto* bk = reinterpret_cast<unsigned*>(descale_k);
+  auto* bv = reinterpret_cast<unsigned*>(descale_v);
+  const dim3 gq(std::max(1, std::min((total_tokens + 31) / 32, grid / hq + 1)), hq);
+  const dim3 gk(std::max(1, std::min((total_tokens + 31) / 32, grid / hkv + 1)), hkv);
+  launch(amax_per_head, gq, qb, total_tokens, hq, d, bq);
+  launch(amax_per_head, gk, kb, total_tokens, hkv, d, bk);
+  launch(amax_per_head, gk, vb, total_tokens, hkv, d, bv);
+  launch(amax_to_descale, dim3((hq + 255) / 256), bq, hq);
+  launch(amax_to_descale, dim3((hkv + 255) / 256), bk, hkv);
+  launch(amax_to_descale, dim3((hkv + 255) / 256), bv, hkv);
+  launch(quantize_rows, dim3(grid), qb, nq, hq, d, static_cast<const float*>(descale_q), static_cast<uint8_t*>(q8));
+  launch(quantize_rows, dim3(grid), kb, nk, hkv, d, static_cast<const float*>(descale_k), static_cast<uint8_t*>(k8));
+  launch(quantize_v_transposed, dim3((pitch + 63) / 64, d / 64, batch * hkv), vb, seqlen, pitch, hkv, d,
+         static_cast<const float*>(descale_v), static_cast<uint8_t*>(vt8));
+  e = cudaGetLastError();
   return e;
 }
 
