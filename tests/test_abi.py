@@ -157,3 +157,22 @@ def test_fp8_calls_reject_bad_arguments_on_host(lib):
     assert lib.attn_fp8_quantize(p, p, p, 1, 64, 2, 2, 128, p, None, p, p, p, p, None) == attn.ATTN_ERR_INVALID_ARG
     assert lib.attn_fp8_quantize(None, None, None, 0, 64, 2, 2, 128, None, None, None, None, None, None,
                                  None) == attn.ATTN_OK
+
+
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    """include/attn.h is a C header (C99, no C++), and a C program links libattn.so and
+    gets the host-side answers (workspace sizes, validation statuses) without a GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(attn.LIBRARY_PATH)
+    exe = str(tmp_path / "c_abi_client")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_abi_client.c"), "-o", exe, "-L", libdir, "-lattn",
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert "unsupported configuration" in r.stdout and "invalid argument" in r.stdout
