@@ -25,17 +25,17 @@
 //                         dV  += P^T dO_i             (A from TMEM)
 //                         dK  += dS^T Q_i             (A from TMEM)
 //                         dQ_i partial                (A, B from SMEM)
-//                       and a drain warpgroup adds each dQ_i partial into the fp32
-//                       accumulator with fp32 atomics (L2 reductions), reading it from a
-//                       double-buffered TMEM slot so the tensor core never waits on it.
+//                       and a drain warpgroup reads each dQ_i partial out of TMEM, stages
+//                       it in an fp32 SMEM tile and adds it into the fp32 accumulator with
+//                       a bulk tensor reduction (cp.reduce.async.bulk.tensor, in L2).
 //   3. bwd_dq_convert   dQ = bf16(scale * accumulator) (HBM-bound).
 //
 // dQ strategy.  Each (key tile, query tile) pair contributes a BM x d partial of dQ_i;
-// the CTA that owns the key tile adds it into an fp32 accumulator with atomics.  The
+// the CTA that owns the key tile adds it into an fp32 accumulator (reductions in L2).  The
 // alternative -- a second, query-major kernel -- would recompute S and dP (7 matrix
-// products per tile instead of 5, 40% more tensor work); the atomic traffic instead goes
-// to L2 (the accumulator of one head, N*d*4 bytes, stays L2-resident): the drain stages
-// each partial in an fp32 SMEM tile and adds it with bulk tensor reductions.
+// products per tile instead of 5, 40% more tensor work); the reduction traffic instead
+// goes to L2 (the accumulator of one head, N*d*4 bytes, stays L2-resident): the drain
+// stages each partial in an fp32 SMEM tile and adds it with bulk tensor reductions.
 //
 // TMEM shapes.  d = 128 uses BM = 64 query rows per step and forms the transpose
 // dQ_i^T = K_j^T dS^T (M = d = 128, N = 64), which fits S^T (64) + dP^T (64) + dV (128)

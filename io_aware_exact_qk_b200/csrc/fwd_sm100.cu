@@ -25,11 +25,12 @@
 //
 // Persistent schedule: one CTA per SM claims work items from a global counter in a fixed
 // order -- heaviest first under the causal mask, within groups of heads whose K/V fit in
-// L2; pairs of one head adjacent otherwise (their K/V stream is shared through L2).  All
-// pipelines run
-// across items: the next item's Q load and its first QK^T MMAs overlap the current item's
-// epilogue, and the K/V ring never drains.  Under the causal mask a query tile only
-// visits key tiles it can see, so the lower tile of an item skips the last key tile.
+// L2; pairs of one head adjacent otherwise (their K/V stream is shared through L2), with
+// a last wave that would leave most SMs idle split into single-tile items.  All pipelines
+// run across items: each Q tile buffer reloads as soon as its own last QK^T is done, the
+// next item's first QK^T MMAs overlap the current item's epilogue, and the K/V ring never
+// drains.  Under the causal mask a query tile only visits key tiles it can see, so the
+// lower tile of an item skips the last key tile.
 //
 // Warp roles (320 threads):
 //   warps 0-3  softmax + correction + epilogue for query tile 0 (TMEM lanes 0..127)
