@@ -200,10 +200,21 @@ def max_over_ranks(ms, world, device):
 # ---------------------------------------------------------------------------------------
 # GPU side
 # ---------------------------------------------------------------------------------------
+def code_hash(path):
+    """sha256 (first 16 hex digits) of a C/CUDA source with its comments and all whitespace
+    removed: it changes when the code does, not when only a comment is edited."""
+    import hashlib
+    import re
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    text = re.sub(r"\s+", "", text)
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
 def traffic_record(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
-    import hashlib
+    the current kernel code (else None)."""
     path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
     if not os.path.exists(path):
         return None
@@ -212,8 +223,7 @@ def traffic_record(kernel):
     if not rec:
         return None
     src = os.path.join(ROOT, "io_aware_exact_qk_b200", "csrc", rec["source"])
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+    return rec["dram_bytes_per_launch"] if code_hash(src) == rec["source_code_sha256_16"] else None
 
 
 def run_ours(args, rank, world, local_rank):
