@@ -67,7 +67,7 @@ extern "C" {
 typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_INVALID_ARG = 1,   /* a pointer, size or shape argument is invalid          */
-    ATTN_ERR_UNSUPPORTED = 2,   /* valid but outside what this build supports (d, dtype) */
+    ATTN_ERR_UNSUPPORTED = 2,   /* valid but outside what this library supports (d, dtype) */
     ATTN_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed                  */
     ATTN_ERR_TIMEOUT = 4        /* a kernel's bounded pipeline wait ran out              */
 } attn_status;

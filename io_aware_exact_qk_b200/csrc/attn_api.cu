@@ -76,7 +76,7 @@ attn_status check_shapes(const int32_t* cu_seqlens, int32_t batch, int32_t seqle
   }
   // TMA row coordinates and the [hq, T] statistics are addressed with 32-bit rows.
   if ((int64_t)total_tokens * hq > (int64_t)INT32_MAX * 4)
-    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
   pb->cu_seqlens = cu_seqlens;
   pb->batch = batch;
   pb->seqlen = cu_seqlens ? 0 : seqlen;
@@ -225,10 +225,10 @@ attn_status check_fp8(int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, in
                       Problem* pb) {
   if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 forward needs head dim 64 or 128 (got %d)", d);
   if (batch < 0 || seqlen < 0) return fail(ATTN_ERR_INVALID_ARG, "negative batch / seqlen");
-  if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+  if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
   if ((int64_t)batch * hkv > 65535) return fail(ATTN_ERR_UNSUPPORTED, "batch * hkv must be <= 65535");
   if ((int64_t)batch * hkv * d * fp8_vt_pitch(seqlen) > ((int64_t)1 << 40))
-    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
   return check_shapes(nullptr, batch, seqlen, seqlen, batch * seqlen, hq, hkv, d, scale, causal, ATTN_BF16, pb);
 }
 }  // namespace
@@ -334,7 +334,7 @@ attn_status check_decode(const int32_t* cu_q, const int32_t* cu_k, int32_t batch
     return fail(ATTN_ERR_UNSUPPORTED, "(hq / hkv) * max_seqlen_q = %lld exceeds 128 query rows per KV head",
                 (long long)(hq / hkv) * max_seqlen_q);
   if ((int64_t)total_q * hq > (int64_t)INT32_MAX || (int64_t)total_k * hkv > (int64_t)INT32_MAX * 4)
-    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this build");
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
   pb->cu_q = cu_q;
   pb->cu_k = cu_k;
   pb->batch = batch;

@@ -7,9 +7,8 @@ every rank the hops of ``ring_schedule`` are executed with the library's kernels
 and the rows of all ranks together must match the fp64 oracle over the whole sequences
 with the forward's tolerances; the backward's per-hop gradients, summed the way the
 travelling dK / dV are, must match the oracle's gradient at the backward's tolerance.
-The point-to-point passing of the blocks between real
-ranks is covered by the gloo test on the CPU; the driver itself runs here as a one-rank
-NCCL group.
+The point-to-point passing of the blocks between real ranks is covered by the gloo test
+on the CPU; the ring functions themselves run here as a one-rank NCCL group.
 """
 import datetime
 import socket
@@ -130,7 +129,7 @@ def test_merge_kernel_edge_cases():
 
 
 def test_driver_as_a_one_rank_nccl_group():
-    """The driver's own code path (defaults = the library's kernels) on one rank."""
+    """The ring functions' own code path (defaults = the library's kernels) on one rank."""
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
