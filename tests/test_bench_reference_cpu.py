@@ -44,3 +44,20 @@ def test_warmup_below_three_is_refused():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
                        capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert r.returncode != 0
+
+
+def test_traffic_record_follows_the_code_not_the_comments(tmp_path):
+    """bench.py reports an ncu traffic figure only while the kernel's code is the one the
+    counters were taken on: comment and whitespace edits keep the hash, code edits do not."""
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("// header\n__global__ void k(int* p) {\n  p[0] = 1;  /* store */\n}\n")
+    h0 = bench.code_hash(str(src))
+    src.write_text("// a longer header\n// over two lines\n__global__ void k(int* p) {\n    p[0] = 1;\n}\n")
+    assert bench.code_hash(str(src)) == h0
+    src.write_text("__global__ void k(int* p) {\n  p[0] = 2;\n}\n")
+    assert bench.code_hash(str(src)) != h0
+    # the committed records: the backward's matches its current source
+    assert bench.traffic_record("bwd_bf16_sm100") is not None
+    assert bench.traffic_record("no_such_kernel") is None

@@ -83,3 +83,19 @@ def test_rounding_changes_the_output_by_a_bounded_amount():
     o2, _ = oracle.attn_fwd_fp8sim(q, k, v, causal=True, round_p=False)
     err = np.abs(o - o2).max()
     assert 0 < err <= 2 ** -4 * np.abs(v).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rounded_weights_leave_the_lse_exact(causal):
+    """The row sum is formed from the unrounded weights, so with the rounding on the LSE
+    is still the exact one (the rounding only touches the weighted sum of V)."""
+    rng = np.random.default_rng(7)
+    cu = np.array([0, 260, 700])
+    hq, hkv, d = 2, 1, 32
+    q = rng.standard_normal((700, hq, d)) * 2.0
+    k = rng.standard_normal((700, hkv, d)) * 2.0
+    v = rng.standard_normal((700, hkv, d))
+    o, lse = oracle.attn_fwd_fp8sim(q, k, v, cu, causal=causal, round_p=True)
+    o2, lse2 = oracle.attn_fwd(q, k, v, cu, causal=causal)
+    np.testing.assert_allclose(lse, lse2, rtol=1e-14, atol=1e-11)
+    assert np.abs(o - o2).max() > 1e-6          # while O does move with the rounding

@@ -64,6 +64,7 @@ def _battery():
         lambda: dpins.test_cross_zero_queries_average_the_visible_values(),
         lambda: fpins.test_two_key_example_rounds_the_weights_but_not_the_sum(),
         lambda: fpins.test_unrounded_steps_equal_the_exact_forward(True, 30.0),
+        lambda: fpins.test_rounded_weights_leave_the_lse_exact(True),
     ]
     for c in checks:
         try:
