@@ -1,20 +1,23 @@
 #!/usr/bin/env python
 """Throughput of the exact-attention hot path (forward + backward) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 A step is one pass of the whole hot path over one batch of synthetic input: attn_fwd and
-attn_bwd (D preprocess, main backward, dQ convert) on the multi-head workload
-B=4, H=16, N=2048, d=128, bf16, once without and once with the causal mask.  The metric is
-attention TFLOP/s (4*B*H*N^2*d for the forward, 2.5x that for the backward, halved for
-causal) and its fraction of the measured dense BF16 tensor-core peak.
+attn_bwd (D preprocess, main backward, dQ convert) on the gate workload B=4, H=16,
+N=4096, d=128, bf16 (the head_dim/seqlen sweep's d=128, N=4096 point), once without and
+once with the causal mask.  The metric is attention TFLOP/s (4*B*H*N^2*d for the forward,
+2.5x that for the backward, halved for causal) and its fraction of the measured dense
+BF16 tensor-core peak; the line also gives the forward and the backward pass separately
+(per mask), each with the roofline of its main kernel and the oracle's time for the same
+pass.
 
 One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE); each rank runs its own
 batch (weak scaling, no collective on the data path); the time is the max over ranks.
-Timing: CUDA events on the launching stream around each step, L2 flushed (a 256 MiB
-write) between timed steps, per-kernel times from the library's own launch events.
-``--impl reference`` times the fp64 CPU oracle (the only reference there is) on a bounded
-sample of the same workload, on rank 0 only.
+Timing: CUDA events on the launching stream around each step and each pass, L2 flushed
+(a 256 MiB write) between timed steps, per-kernel times from the library's own launch
+events.  ``--impl reference`` times the fp64 CPU oracle (the only reference there is) on
+a bounded sample of the same workload, on rank 0 only.
 """
 import argparse
 import dataclasses
@@ -39,7 +42,8 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 DATA = "synthetic: Q, K, V, dO iid N(0,1) drawn in fp32 from a seeded torch CPU generator, rounded to bf16"
 
 
-WORKLOAD = "mha2k"   # set from --workload
+DEFAULT_WORKLOAD = "sweep_d128_n4096"
+WORKLOAD = DEFAULT_WORKLOAD   # set from --workload
 
 
 def base_workload(name):
@@ -138,9 +142,10 @@ _ORACLE_CACHE = {}
 def oracle_sample(heads, budget_s=None):
     """Oracle forward + backward on whole heads of sequence 0 of both variants.  Runs the
     given number of heads, or (budget_s) adds heads until the budget is spent.
-    Returns (algorithmic flops, seconds, heads done, threads)."""
+    Returns ({"fwd": (flops, s), "bwd": (flops, s)}, heads done, threads)."""
     import oracle
-    flops, secs, done = 0.0, 0.0, 0
+    per = {"fwd": [0.0, 0.0], "bwd": [0.0, 0.0]}
+    done = 0
     threads = oracle.default_threads()
     variants = workload_variants()
     base = variants[0]
@@ -152,19 +157,27 @@ def oracle_sample(heads, budget_s=None):
     for h in range(base.hq):
         if heads is not None and done >= heads:
             break
-        if budget_s is not None and secs >= budget_s:
+        if budget_s is not None and per["fwd"][1] + per["bwd"][1] >= budget_s:
             break
         qs, dos = (t[:n, h:h + 1].contiguous() for t in (q, do))
         ks, vs = (t[:n, h // G:h // G + 1].contiguous() for t in (k, v))
         for causal in sorted({w.causal for w in variants}):
+            f = 4.0 * n * n * base.d * (0.5 if causal else 1.0)
             t0 = time.perf_counter()
             oracle.attn_fwd(qs, ks, vs, scale=base.scale, causal=causal, threads=threads)
+            t1 = time.perf_counter()
             oracle.attn_bwd(qs, ks, vs, dos, scale=base.scale, causal=causal, threads=threads)
-            secs += time.perf_counter() - t0
-            f = 4.0 * n * n * base.d * (0.5 if causal else 1.0)
-            flops += 3.5 * f
+            t2 = time.perf_counter()
+            per["fwd"][0] += f
+            per["fwd"][1] += t1 - t0
+            per["bwd"][0] += 2.5 * f
+            per["bwd"][1] += t2 - t1
         done += 1
-    return flops, secs, done, threads
+    return {k_: tuple(v_) for k_, v_ in per.items()}, done, threads
+
+
+def oracle_totals(per):
+    return per["fwd"][0] + per["bwd"][0], per["fwd"][1] + per["bwd"][1]
 
 
 def run_reference(args, rank, world):
@@ -175,7 +188,8 @@ def run_reference(args, rank, world):
     flops = secs = 0.0
     threads = 1
     for _ in range(args.steps):
-        f, s, _, threads = oracle_sample(heads=1)
+        per, _, threads = oracle_sample(heads=1)
+        f, s = oracle_totals(per)
         flops += f
         secs += s
     value = flops / secs / 1e12
@@ -212,18 +226,39 @@ def code_hash(path):
     return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
-def traffic_record(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
-    the current kernel code (else None)."""
-    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+def traffic_record(kernel, workload=None, path=None):
+    """The committed ncu record of `kernel` (DRAM bytes per launch, tensor-pipe and
+    special-function-unit activity) if it was taken on the current kernel code and, when
+    `workload` is given, on that workload (else None: the figures would not apply).
+    Records are keyed "<kernel>@<workload>"."""
+    path = path or os.path.join(ROOT, "profiles", "roofline_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(kernel)
-    if not rec:
+        table = json.load(f)
+    if workload is not None:
+        rec = table.get(f"{kernel}@{workload}")
+    else:
+        rec = next((r for key, r in table.items() if key.split("@")[0] == kernel), None)
+    if not isinstance(rec, dict):
         return None
     src = os.path.join(ROOT, "io_aware_exact_qk_b200", "csrc", rec["source"])
-    return rec["dram_bytes_per_launch"] if code_hash(src) == rec["source_code_sha256_16"] else None
+    return rec if code_hash(src) == rec["source_code_sha256_16"] else None
+
+
+def roofline_block(kernel, flops_per_launch, mean_launch_ms, peaks, workload):
+    """Roofline of one tensor-bound kernel: algorithmic FLOPs per launch over its mean
+    event-timed launch, against the measured dense bf16 peak; DRAM traffic and ncu's
+    tensor-pipe activity from the committed capture of the same code and workload."""
+    achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
+    rec = traffic_record(kernel, workload)
+    return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": UNIT,
+            "frac": achieved / peaks["bf16_tflops"],
+            "traffic": rec["dram_bytes_per_launch"] if rec else None,
+            "ncu_tensor_pipe_active": rec.get("tensor_pipe_active") if rec else None,
+            "ncu_sfu_pipe_active": rec.get("xu_pipe_active") if rec else None,
+            "peak_source": f"{peaks['source']} dense bf16 (burst)",
+            "flops_per_launch": flops_per_launch, "mean_launch_ms": mean_launch_ms}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -245,12 +280,20 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def step(marks=None):
+        """One step; with `marks` ({(causal, pass): [start, end] events}) each pass is
+        bracketed by events on the launching stream."""
         for w in variants:
             b = outs[w.causal]
+            if marks:
+                marks[(w.causal, "fwd")][0].record(stream)
             attn.attn_fwd(qd, kd, vd, scale=w.scale, causal=w.causal, o=b["o"], lse=b["lse"], **shape_kw)
+            if marks:
+                marks[(w.causal, "fwd")][1].record(stream)
             attn.attn_bwd(qd, kd, vd, b["o"], dod, b["lse"], scale=w.scale, causal=w.causal,
                           dq=b["dq"], dk=b["dk"], dv=b["dv"], workspace=ws, **shape_kw)
+            if marks:
+                marks[(w.causal, "bwd")][1].record(stream)
 
     def barrier():
         if world > 1:
@@ -265,33 +308,47 @@ def run_ours(args, rank, world, local_rank):
     attn.attn_get_device_error()
     barrier()
 
-    # ---- timed region (device): per-step events, L2 flushed between steps ----
+    # ---- timed region (device): per-step and per-pass events, L2 flushed between steps ----
+    def new_marks():
+        m = {}
+        for w in variants:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            m[(w.causal, "fwd")] = (e[0], e[1])
+            m[(w.causal, "bwd")] = (e[1], e[2])   # the backward starts where the forward ends
+        return m
+
     attn.attn_profile_collect()
     attn.attn_profile_enable(True)
     launches0 = attn.attn_launch_count()
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), new_marks())
+              for _ in range(args.steps)]
     with ClockSampler(local_rank) as clocks:
         barrier()
-        for s, e in events:
+        for s, e, marks in events:
             flush.zero_()
             s.record(stream)
-            step()
+            step(marks)
             e.record(stream)
         barrier()
     attn.attn_profile_enable(False)
     launches = attn.attn_launch_count() - launches0
     per_kernel = attn.attn_profile_collect()
     attn.attn_get_device_error()
-    total_ms = sum(s.elapsed_time(e) for s, e in events)
+    total_ms = sum(s.elapsed_time(e) for s, e, _ in events)
     total_ms = max_over_ranks(total_ms, world, dev)
     value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+    pass_ms = {key: max_over_ranks(sum(m[key][0].elapsed_time(m[key][1]) for _, _, m in events), world, dev)
+               for key in events[0][2]}
 
     # ---- end to end: host buffers, copies inside the timed region ----
     if args.quick:
         if rank == 0:
             print(json.dumps({"quick": True, "value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
+                              "passes_ms": {f"{p_}{'+causal' if c else ''}": v_ / args.steps
+                                            for (c, p_), v_ in pass_ms.items()},
                               "kernels": {k: list(v) for k, v in per_kernel.items()}, "gpu_launches": launches}))
         return
+    e2e_steps = min(args.steps, 20)
     e2e_bufs = {}
     e2e_out = {}
     host_kw = dict(cu_seqlens=cu, max_seqlen=w0.max_seqlen) if w0.varlen else dict(batch=w0.batch)
@@ -305,7 +362,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_start, e2e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_start.record(stream)
-    for _ in range(args.steps):
+    for _ in range(e2e_steps):
         for w in variants:
             e2e_out[w.causal], _ = attn.attention_host(host["q"], host["k"], host["v"], host["do"], scale=w.scale,
                                                        causal=w.causal, out=e2e_bufs[w.causal], **host_kw)
@@ -313,38 +370,68 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     attn.attn_get_device_error()
     e2e_ms = e2e_start.elapsed_time(e2e_end)
-    e2e_value = world * flops_step * args.steps / (max_over_ranks(e2e_ms, world, dev) / 1e3) / 1e12
+    e2e_value = world * flops_step * e2e_steps / (max_over_ranks(e2e_ms, world, dev) / 1e3) / 1e12
 
     if rank != 0:
         return
     peaks = load_peaks()
+    # per-pass results: TF/s of each (pass, mask) from its events, and the roofline of the
+    # pass's main kernel from the library's per-launch events
+    cpu = None
+    cpu_per = None
+    if world == 1:
+        cpu_per, heads, threads = oracle_sample(heads=None, budget_s=12.0)
+        f, s_ = oracle_totals(cpu_per)
+        cpu = {"value": f / s_ / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 CPU oracle, fwd+bwd of {heads} whole head(s) of sequence 0 of {WORKLOAD} "
+                         f"(all its mask variants), {s_:.1f} s"}
+    passes = {}
+    for pname, kname, mult in (("fwd", "fwd_bf16_sm100", 1.0), ("bwd", "bwd_bf16_sm100", 2.5)):
+        by_mask = {}
+        tot_f = tot_ms = 0.0
+        for w in variants:
+            f = mult * flops_fwd[w.causal] * args.steps
+            ms = pass_ms[(w.causal, pname)]
+            by_mask["causal" if w.causal else "non_causal"] = {
+                "value": world * f / (ms / 1e3) / 1e12, "frac": world * f / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                "ms": ms / args.steps}
+            tot_f += f
+            tot_ms += ms
+        entry = {"value": world * tot_f / (tot_ms / 1e3) / 1e12, "unit": UNIT,
+                 "frac": world * tot_f / (tot_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                 "ms_per_step": tot_ms / args.steps, "by_mask": by_mask,
+                 "includes": ("attn_fwd: work-item counter reset + fwd_bf16_sm100" if pname == "fwd" else
+                              "attn_bwd: bwd_preprocess + bwd_bf16_sm100 + bwd_dq_convert")}
+        if kname in per_kernel:
+            k_ms, k_n = per_kernel[kname]
+            entry["roofline"] = roofline_block(kname, mult * sum(flops_fwd.values()) * args.steps / k_n,
+                                               k_ms / k_n, peaks, WORKLOAD)
+        if cpu_per is not None:
+            f, s_ = cpu_per[pname]
+            entry["cpu_baseline"] = {"value": f / s_ / 1e12, "unit": UNIT, "cores": cpu["cores"], "kind": "oracle",
+                                     "sample": f"fp64 CPU oracle, {pname} of {heads} whole head(s) of sequence 0 of "
+                                               f"{WORKLOAD} (all its mask variants), {s_:.1f} s"}
+        passes[pname] = entry
     # dominant kernel and its roofline (algorithmic FLOPs per launch / mean event duration)
     dom = max(per_kernel, key=lambda n: per_kernel[n][0])
     dom_ms, dom_n = per_kernel[dom]
     if dom.startswith("bwd_bf16"):
         dom_flops = sum(2.5 * f for f in flops_fwd.values()) * args.steps
-    else:
+    elif dom.startswith("fwd_bf16"):
         dom_flops = sum(flops_fwd.values()) * args.steps
-    achieved = dom_flops / (dom_ms / 1e3) / 1e12
-    traffic = traffic_record(dom)
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": UNIT,
-                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_source": f"{peaks['source']} dense bf16 (burst)",
-                "flops_per_launch": dom_flops / dom_n, "mean_launch_ms": dom_ms / dom_n}
+    else:
+        dom_flops = 0.0
+    roofline = roofline_block(dom, dom_flops / dom_n, dom_ms / dom_n, peaks, WORKLOAD)
     breakdown = {}
     for name, (ms, n) in sorted(per_kernel.items()):
         breakdown[name] = {"launches": n, "total_ms": ms, "share": ms / sum(x[0] for x in per_kernel.values())}
-    cpu = None
-    if world == 1:
-        f, s, heads, threads = oracle_sample(heads=None, budget_s=12.0)
-        cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"fp64 CPU oracle, fwd+bwd of {heads} whole head(s) of sequence 0 of {WORKLOAD} "
-                         f"(all its mask variants), {s:.1f} s"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config_block(world),
-            "pct_of_peak": value / peaks["bf16_tflops"], "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "pct_of_peak": value / peaks["bf16_tflops"], "roofline": roofline, "passes": passes,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
             "gpu_launches": launches, "clocks": clocks.summary(), "kernels": breakdown}
     print(json.dumps(line), flush=True)
 
@@ -690,11 +777,12 @@ def run_fp8(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha2k",
-                    help="mha2k (the metric's configuration), sweep_d<d>_n<N>, gqa8k, varlen16, long32k; "
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="sweep_d128_n4096 (default: the gate's d=128, N=4096 point), mha2k, sweep_d<d>_n<N>, "
+                         "gqa8k, varlen16, long32k; "
                          "or a split-KV decode workload: decode8k, decode_var, decode_spec4; "
                          "or the FP8 forward: fp8_mha2k")
     ap.add_argument("--quick", action="store_true",

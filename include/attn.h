@@ -247,6 +247,34 @@ const char *attn_profile_kernel_name(int32_t kind);
 attn_status attn_profile_collect(double *total_ms, int64_t *launches, int32_t n);
 int64_t attn_launch_count(void);
 
+/* ---- failure detection and self-tests -------------------------------------------------
+ * Every pipeline wait inside the library's kernels is bounded in wall time.  A wait that
+ * runs out marks its CTA aborted (the CTA's other roles stop waiting), records a timeout in
+ * the device error word and lets the kernel return, so a broken pipeline ends as
+ * ATTN_ERR_TIMEOUT from attn_get_device_error() instead of a hung GPU.  (The pages define no
+ * such mechanism; it is this library's failure detection.)
+ *
+ * attn_set_wait_limit_ns sets the bound for the CURRENT device, in nanoseconds (default
+ * 2 000 000 000, 2 s; 0 is ATTN_ERR_INVALID_ARG); attn_get_wait_limit_ns reads it (0 if the
+ * read failed).  It is a per-device global that kernels read while they wait: change it
+ * between calls, not while the library's kernels run.  A limit far below a kernel's normal
+ * waits (a few microseconds) turns ordinary waits into timeouts.
+ *
+ * attn_selftest_wait launches one CTA that waits on a barrier with that same bounded wait.
+ * arrive = 1: the barrier completes and the wait returns at once.  arrive = 0: nothing
+ * arrives, the wait runs out after the limit and attn_get_device_error() reports
+ * ATTN_ERR_TIMEOUT; the CTA holds no copy, MMA or Tensor Memory when it gives up, and the
+ * GPU stays usable.  Asynchronous on `stream`.
+ *
+ * attn_selftest_exp2 writes, for n floats x (device pointers, 4-byte aligned), y_fma[i] =
+ * the forward kernel's FMA-pipe evaluation of 2^x[i] and y_sfu[i] = the special-function
+ * unit's approximate 2^x[i], so that the former can be checked against its error bound
+ * (relative error below 7.6e-5 for x in [-125, 8]; 7.51e-5 at worst).  Asynchronous on `stream`. */
+attn_status attn_set_wait_limit_ns(uint64_t ns);
+uint64_t attn_get_wait_limit_ns(void);
+attn_status attn_selftest_wait(int32_t arrive, void *stream);
+attn_status attn_selftest_exp2(const float *x, float *y_fma, float *y_sfu, int64_t n, void *stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int32_t attn_version(void);
 

@@ -83,6 +83,14 @@ def load_library():
     lib.attn_fp8_quantize.restype = ctypes.c_int
     lib.attn_fwd_fp8.argtypes = [vp] * 6 + [i32] * 5 + [f32, i32, vp, vp, vp, sz, vp]
     lib.attn_fwd_fp8.restype = ctypes.c_int
+    lib.attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.attn_set_wait_limit_ns.restype = ctypes.c_int
+    lib.attn_get_wait_limit_ns.argtypes = []
+    lib.attn_get_wait_limit_ns.restype = ctypes.c_uint64
+    lib.attn_selftest_wait.argtypes = [i32, vp]
+    lib.attn_selftest_wait.restype = ctypes.c_int
+    lib.attn_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
+    lib.attn_selftest_exp2.restype = ctypes.c_int
     lib.attn_launch_count.argtypes = []
     lib.attn_launch_count.restype = ctypes.c_int64
     _lib = lib
@@ -309,6 +317,30 @@ def attn_fwd_fp8(q8, k8, vt8, descale_q, descale_k, descale_v, batch, scale=None
 def attn_get_device_error(stream=None):
     """Synchronise the stream and raise if a kernel reported a device-side error."""
     _check(load_library().attn_get_device_error(_stream(stream)))
+
+
+def attn_set_wait_limit_ns(ns):
+    """Bound (ns of wall time) on every pipeline wait of the library's kernels, current device."""
+    _check(load_library().attn_set_wait_limit_ns(int(ns)))
+
+
+def attn_get_wait_limit_ns():
+    return int(load_library().attn_get_wait_limit_ns())
+
+
+def attn_selftest_wait(arrive, stream=None):
+    """One CTA waits on a barrier with the library's bounded wait; without `arrive` the wait
+    runs out and attn_get_device_error() raises with ATTN_ERR_TIMEOUT."""
+    _check(load_library().attn_selftest_wait(int(bool(arrive)), _stream(stream)))
+
+
+def attn_selftest_exp2(x, stream=None):
+    """(y_fma, y_sfu): the forward's FMA-pipe 2^x and the special-function unit's 2^x of the
+    float32 device tensor x."""
+    x = x.contiguous()
+    y_fma, y_sfu = torch.empty_like(x), torch.empty_like(x)
+    _check(load_library().attn_selftest_exp2(_ptr(x), _ptr(y_fma), _ptr(y_sfu), x.numel(), _stream(stream)))
+    return y_fma, y_sfu
 
 
 def attn_version():

@@ -16,6 +16,7 @@
 namespace attn {
 
 __device__ uint32_t g_device_error = 0;
+__device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 
 namespace {
 
@@ -128,7 +129,7 @@ const char* kernel_kind_name(int kind) {
                                            "bwd_dq_convert",  "fwd_fp32_kernel",      "bwd_fp32_dq_kernel",
                                            "bwd_fp32_dkdv_kernel", "decode_bf16_sm100", "decode_combine",
                                            "merge_partial",   "merge_finish",         "fwd_fp8_sm100",
-                                           "fp8_quantize"};
+                                           "fp8_quantize",    "selftest"};
   return (kind >= 0 && kind < K_NUM_KINDS) ? names[kind] : "";
 }
 
@@ -449,20 +450,39 @@ size_t attn_bwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_
   return dtype == ATTN_FP32 ? bwd_fp32_workspace_bytes(pb) : bwd_bf16_workspace_bytes(pb);
 }
 
-attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                     const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
-                     int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
-                     int32_t dtype, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                     void* stream) {
-  Problem pb;
+}  // extern "C"
+
+namespace attn {
+// Host validation of the backward's arguments (shapes, then tensor pointers when there is
+// work to do); touches no GPU state.
+int bwd_check_args(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                   int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                   int32_t dtype, void* dq, void* dk, void* dv, Problem* pb) {
   attn_status st = check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal,
-                                dtype, &pb);
+                                dtype, pb);
   if (st != ATTN_OK) return st;
   if (total_tokens == 0 || batch == 0) return ok();
   if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
       (st = check_ptr(o, "o")) || (st = check_ptr(dout, "dout")) || (st = check_ptr(lse, "lse")) ||
       (st = check_ptr(dq, "dq")) || (st = check_ptr(dk, "dk")) || (st = check_ptr(dv, "dv")))
     return st;
+  return ok();
+}
+}  // namespace attn
+
+extern "C" {
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                     int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                     int32_t dtype, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  Problem pb;
+  attn_status st = (attn_status)bwd_check_args(q, k, v, o, dout, lse, cu_seqlens, batch, seqlen, max_seqlen,
+                                               total_tokens, hq, hkv, d, scale, causal, dtype, dq, dk, dv, &pb);
+  if (st != ATTN_OK) return st;
+  if (total_tokens == 0 || batch == 0) return ok();
   const size_t need = attn_bwd_workspace_size(batch, pb.max_seqlen, total_tokens, hq, hkv, d, dtype);
   if (workspace_bytes < need)
     return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
@@ -488,6 +508,33 @@ attn_status attn_get_device_error(void* stream) {
   if (word & ATTN_DEVERR_TIMEOUT) return fail(ATTN_ERR_TIMEOUT, "a kernel's pipeline wait timed out");
   if (word & ATTN_DEVERR_SEQLEN) return fail(ATTN_ERR_INVALID_ARG, "a sequence is longer than max_seqlen");
   return ok();
+}
+
+attn_status attn_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return fail(ATTN_ERR_INVALID_ARG, "the wait limit must be positive");
+  const cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof ns);
+  return from_cuda(e, "setting the wait limit");
+}
+
+uint64_t attn_get_wait_limit_ns(void) {
+  uint64_t ns = 0;
+  if (cudaMemcpyFromSymbol(&ns, g_wait_limit_ns, sizeof ns) != cudaSuccess) return 0;
+  return ns;
+}
+
+attn_status attn_selftest_wait(int32_t arrive, void* stream) {
+  if (arrive != 0 && arrive != 1) return fail(ATTN_ERR_INVALID_ARG, "arrive must be 0 or 1");
+  return from_cuda(launch_selftest_wait(arrive, static_cast<cudaStream_t>(stream)), "selftest launch");
+}
+
+attn_status attn_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int64_t n, void* stream) {
+  if (n < 0) return fail(ATTN_ERR_INVALID_ARG, "negative element count");
+  if (n == 0) return ok();
+  if (x == nullptr || y_fma == nullptr || y_sfu == nullptr)
+    return fail(ATTN_ERR_INVALID_ARG, "x, y_fma and y_sfu must be device pointers");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y_fma) | reinterpret_cast<uintptr_t>(y_sfu)) & 3u)
+    return fail(ATTN_ERR_INVALID_ARG, "x, y_fma and y_sfu must be 4-byte aligned");
+  return from_cuda(launch_selftest_exp2(x, y_fma, y_sfu, n, static_cast<cudaStream_t>(stream)), "selftest launch");
 }
 
 const char* attn_status_string(attn_status status) {

@@ -270,6 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (threadIdx.x == 0) {
+    // Key tiles past max_seqlen are not in the item list, so a longer sequence would lose
+    // part of its gradients: report it (the items still run, on the tiles they cover).
+    if (blockIdx.x == 0)
+      for (int b = 0; b < p.batch; ++b) {
+        const int len = p.cu_seqlens ? p.cu_seqlens[b + 1] - p.cu_seqlens[b] : p.seqlen;
+        if (len > p.max_seqlen) report_error(ATTN_DEVERR_SEQLEN);
+      }
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
       // warp-level arrivals: one per compute warp (PT, DS, K buffer free, epilogue read

@@ -76,6 +76,11 @@ cudaError_t launch_bwd_fp32(const Problem& pb, const float* q, const float* k, c
                             const float* dout, const float* lse, float* dq, float* dk, float* dv, void* workspace,
                             cudaStream_t stream);
 
+// Diagnostics (diag.cu): a bounded wait that completes (arrive != 0) or runs out, and
+// the forward's FMA-pipe 2^x next to the special-function unit's, element by element.
+cudaError_t launch_selftest_wait(int arrive, cudaStream_t stream);
+cudaError_t launch_selftest_exp2(const float* x, float* y_fma, float* y_sfu, int64_t n, cudaStream_t stream);
+
 // Launch bookkeeping: every kernel launch is wrapped in a LaunchScope, which counts it
 // and, while timing is enabled, brackets it with CUDA events on its stream.
 enum KernelKind : int {
@@ -92,6 +97,7 @@ enum KernelKind : int {
   K_MERGE_FINISH,
   K_FWD_FP8,
   K_FP8_QUANTIZE,
+  K_SELFTEST,
   K_NUM_KINDS
 };
 const char* kernel_kind_name(int kind);
@@ -102,6 +108,13 @@ struct LaunchScope {
   cudaStream_t stream;
   int slot;   // event pair index, -1 when timing is off
 };
+
+// Host validation of attn_bwd's arguments (everything but the workspace); returns an
+// attn_status value and, on failure, records the reason.  Touches no GPU state.
+int bwd_check_args(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                   int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                   int32_t dtype, void* dq, void* dk, void* dv, Problem* pb);
 
 // Records `fmt` as the calling thread's last error message (attn_last_error_message) and
 // returns `status`.

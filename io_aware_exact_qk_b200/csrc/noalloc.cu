@@ -62,19 +62,20 @@ extern "C" attn_status attn_bwd_noalloc(const void* q, const void* k, const void
                                         int32_t batch, int32_t seqlen, int32_t max_seqlen, int32_t total_tokens,
                                         int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
                                         int32_t dtype, void* dq, void* dk, void* dv, void* stream) {
-  // Only a well-formed shape has a meaningful scratch size; anything else goes straight
-  // to attn_bwd's own validation (which fails before touching the GPU).
-  const bool sized = (d == 32 || d == 64 || d == 128) && hq > 0 && hkv > 0 && total_tokens >= 0 &&
-                     (dtype == ATTN_BF16 || dtype == ATTN_FP32);
-  size_t need = 0;
-  if (sized) {
-    need = attn_bwd_workspace_size(batch, cu_seqlens ? max_seqlen : seqlen, total_tokens, hq, hkv, d, dtype);
-    if (need > kNoAllocScratchBytes)
-      return (attn_status)record_error(ATTN_ERR_INVALID_ARG,
-                                       "attn_bwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
-                                       "scratch holds %zu (64 MiB); use attn_bwd with a workspace",
-                                       need, kNoAllocScratchBytes);
-  }
+  // Every argument is checked on the host first, exactly as attn_bwd checks them, so a
+  // malformed call is refused before it touches the GPU (not even the scratch address is
+  // looked up).
+  Problem pb;
+  const int st = bwd_check_args(q, k, v, o, dout, lse, cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv,
+                                d, scale, causal, dtype, dq, dk, dv, &pb);
+  if (st != ATTN_OK) return (attn_status)st;
+  if (total_tokens == 0 || batch == 0) return ATTN_OK;
+  const size_t need = attn_bwd_workspace_size(batch, pb.max_seqlen, total_tokens, hq, hkv, d, dtype);
+  if (need > kNoAllocScratchBytes)
+    return (attn_status)record_error(ATTN_ERR_INVALID_ARG,
+                                     "attn_bwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
+                                     "scratch holds %zu (64 MiB); use attn_bwd with a workspace",
+                                     need, kNoAllocScratchBytes);
   void* scratch = nullptr;
   if (need > 0) {
     const cudaError_t e = scratch_address(&scratch);

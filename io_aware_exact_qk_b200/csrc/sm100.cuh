@@ -2,10 +2,11 @@
 // attention kernels use: mbarriers, TMA tile loads, tcgen05 MMA / TMEM, shared-memory
 // matrix descriptors, plus the per-device error word and bounded waits.
 //
-// Every wait in this library is bounded: a wait that has not completed after
-// kWaitLimitNs of wall time records ATTN_DEVERR_TIMEOUT in the device error word, marks
-// the CTA aborted and returns false, so a broken pipeline ends with an error status
-// instead of a hung GPU.  Kernels never trap.
+// Every wait in this library is bounded: a wait that has not completed after the
+// device's wait limit (g_wait_limit_ns, 2 s unless changed) of wall time records
+// ATTN_DEVERR_TIMEOUT in the device error word, marks the CTA aborted and returns false,
+// so a broken pipeline ends with an error status instead of a hung GPU.  Kernels never
+// trap.
 #pragma once
 
 #include <cuda.h>
@@ -24,9 +25,11 @@ extern __device__ uint32_t g_device_error;
 
 __device__ __forceinline__ void report_error(uint32_t code) { atomicOr(&g_device_error, code); }
 
-// Wall-time bound for one pipeline wait (2 s).  In normal operation every wait is for
-// work inside the same CTA and completes within microseconds.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Wall-time bound for one pipeline wait, per device (default kDefaultWaitLimitNs = 2 s;
+// attn_set_wait_limit_ns changes it between calls).  In normal operation every wait is
+// for work inside the same CTA and completes within microseconds.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+extern __device__ uint64_t g_wait_limit_ns;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -73,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 255u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > *(volatile uint64_t*)&g_wait_limit_ns) {
         *abort_flag = 1;
         report_error(ATTN_DEVERR_TIMEOUT);
         return false;
@@ -307,7 +310,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // n = round(x) obtained by adding 1.5 * 2^23 (which leaves n in the low mantissa bits),
 // f = x - n in [-0.5, 0.5]; 2^f comes from a cubic whose coefficients were fitted to 2^f
 // on [-0.5, 0.5] by least squares on the relative error, reweighted toward the largest
-// errors (max relative error 7.5e-5 in fp32 Horner form); 2^n is applied by adding n to
+// errors (max relative error 7.51e-5 in fp32 Horner form, at f = +-0.5); 2^n is applied by adding n to
 // the exponent field.  Valid for x <= 127 (the softmax passes x <= 8).
 __device__ __forceinline__ void ex2_fma_pair(uint64_t x, float& y0, float& y1) {
   constexpr float kShift = 12582912.0f;          // 1.5 * 2^23

@@ -58,6 +58,20 @@ def test_traffic_record_follows_the_code_not_the_comments(tmp_path):
     assert bench.code_hash(str(src)) == h0
     src.write_text("__global__ void k(int* p) {\n  p[0] = 2;\n}\n")
     assert bench.code_hash(str(src)) != h0
-    # the committed records: the backward's matches its current source
-    assert bench.traffic_record("bwd_bf16_sm100") is not None
-    assert bench.traffic_record("no_such_kernel") is None
+    # a record applies only to its kernel's current code and to its own workload
+    csrc = os.path.join(ROOT, "io_aware_exact_qk_b200", "csrc")
+    table = tmp_path / "records.json"
+    rec = {"source": "bwd_sm100.cu", "source_code_sha256_16": bench.code_hash(os.path.join(csrc, "bwd_sm100.cu")),
+           "dram_bytes_per_launch": 123, "tensor_pipe_active": 0.5}
+    stale = dict(rec, source_code_sha256_16="0" * 16)
+    table.write_text(json.dumps({"bwd_bf16_sm100@wl_a": rec, "fwd_bf16_sm100@wl_a": dict(stale, source="fwd_sm100.cu")}))
+    assert bench.traffic_record("bwd_bf16_sm100", "wl_a", path=str(table))["dram_bytes_per_launch"] == 123
+    assert bench.traffic_record("bwd_bf16_sm100", "wl_b", path=str(table)) is None
+    assert bench.traffic_record("fwd_bf16_sm100", "wl_a", path=str(table)) is None
+    assert bench.traffic_record("no_such_kernel", "wl_a", path=str(table)) is None
+    # every committed record names a source file and the workload it was captured on
+    committed = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))
+    for key, r in committed.items():
+        if key.startswith("_"):
+            continue
+        assert "@" in key and os.path.exists(os.path.join(csrc, r["source"])), key

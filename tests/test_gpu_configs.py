@@ -33,10 +33,21 @@ def _inputs(name, d=None, n=None):
 
 def _run_and_check(w, inputs, picks, seed, **kw):
     out = P.run_full(w, inputs)
-    P.check_sampled(w, inputs, out, picks, seed=seed, tag=w.name, **kw)
+    report = P.check_sampled(w, inputs, out, picks, seed=seed, tag=w.name, **kw)
     P.check_sum_properties(w, inputs[4], inputs[3], out[3], out[4], tag=w.name)
     del out
     torch.cuda.empty_cache()
+    return report
+
+
+# Config 4b against the plain definition (the device's forward and backward, the exact fp64
+# gradients and LSE), measured on B200 over the sampled slices below: max over slices of
+# rel-L2 dQ 1.38e-2, dK 8.4e-3, dV 1.7e-3 and max |LSE - LSE_ref| 1.4e-3.  Stated tolerances:
+# 1e-2 and 1e-3.  dQ and the LSE miss them; the causes are the bf16 rounding of the saved O
+# (through D = rowsum(dO o O), amplified by the cancellation in dP - D when P is nearly
+# one-hot) and fp32 accumulation of scores near 5000 (1e-3 is below two fp32 ulps of the
+# LSE there).  These ceilings catch a regression without pretending the tolerance is met.
+X30_STRICT_CEILING = {"dq": 1.5e-2, "dk": 1e-2, "dv": 1e-2, "lse": 1.5e-3}
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -67,7 +78,12 @@ def test_gqa8k_stability_x30():
         to both the GPU backward (rerun on it) and the oracle's backward -- at the usual
         1e-2."""
     w = W.gqa8k(stability=True)
-    _run_and_check(w, _inputs("gqa8k_x30"), [(0, 0), (1, 7)], seed=8, given=True, fp32_lse_bound_rows=True)
+    report = _run_and_check(w, _inputs("gqa8k_x30"), [(0, 0), (1, 7)], seed=8, given=True,
+                            fp32_lse_bound_rows=True, strict=True)
+    worst = {k: max(r[3][k] for r in report) for k in X30_STRICT_CEILING}
+    print(f"gqa8k_x30 against the exact definition: {worst}")
+    for k, ceiling in X30_STRICT_CEILING.items():
+        assert worst[k] <= ceiling, f"x30 strict {k}: {worst[k]:.3e} above the recorded ceiling {ceiling:.1e}"
 
 
 def test_varlen16():
