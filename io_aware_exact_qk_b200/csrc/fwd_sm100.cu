@@ -601,9 +601,12 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_OFREE + t));
       if (row_ok) {
-        // LSE = m ln 2 + ln l, evaluated in double from the exact fp32 values the
+        // LSE = m ln 2 + ln l, combined in double from the exact fp32 values the
         // exponentials used (m_used, l), minus the first-order effect of scale_log2 being
-        // rounded to fp32 (exact when one score dominates the row), then rounded once.
+        // rounded to fp32 (exact when one score dominates the row), then rounded once.  ln l
+        // itself comes from the fp32 logf (l <= 2^8 * n, so its error is below 1e-6): a
+        // double-precision log is a long software sequence on this path, which every item
+        // boundary waits for.
         // the rounding of the fp32 score factor (for FP8 it includes the two descales)
         double skew = p.lse_skew;
         if constexpr (FP8)
@@ -611,7 +614,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
                  ((double)p.scale_log2 * 0.6931471805599453 - p.lse_skew) * p.descale_q[it.h] * p.descale_k[hk];
         float lse = -INFINITY;
         if (l > 0.f)
-          lse = (float)((double)m_used * 0.6931471805599453 + log((double)l) - skew * (double)mx_used);
+          lse = (float)((double)m_used * 0.6931471805599453 + (double)logf(l) - skew * (double)mx_used);
         p.lse[(size_t)it.h * p.total_tokens + it.seq_start + qi] = lse;
       }
     }

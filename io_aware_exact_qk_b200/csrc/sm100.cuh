@@ -21,15 +21,15 @@ enum : uint32_t {
   ATTN_DEVERR_TIMEOUT = 1u,      // a bounded wait ran out
   ATTN_DEVERR_SEQLEN = 2u,       // a sequence is longer than max_seqlen
 };
-extern __device__ uint32_t g_device_error;
-
-__device__ __forceinline__ void report_error(uint32_t code) { atomicOr(&g_device_error, code); }
-
 // Wall-time bound for one pipeline wait, per device (default kDefaultWaitLimitNs = 2 s;
 // attn_set_wait_limit_ns changes it between calls).  In normal operation every wait is
 // for work inside the same CTA and completes within microseconds.
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+extern __device__ uint32_t g_device_error;
 extern __device__ uint64_t g_wait_limit_ns;
+
+__device__ __forceinline__ void report_error(uint32_t code) { atomicOr(&g_device_error, code); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
