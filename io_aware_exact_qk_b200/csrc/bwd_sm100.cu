@@ -487,6 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         //   NDPT == 1: dP^T(ng+1) here, once dK(ng) has been issued.
         // The first dV / dK of an item overwrite the accumulators, so they wait until the
         // previous item's epilogue has read them out.
+        // Every barrier this thread depends on inside a step is checked with mbar_test one
+        // MMA group before the group that needs it (mbar_wait only if it had not completed
+        // then): the tensor pipe's queue is short, and a check that waits for its own
+        // shared-memory round trip leaves it idle.
+        bool pt_ready = false;   // P^T(ng) seen complete by the check started in the last step
         for (int n = 0; ok && n < w.n_steps; ++n) {
           const int ng = ng0 + n;
           const int s = ng % C::STAGES;
@@ -497,12 +502,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int qslot = C::NDQ == 2 ? b2 : 0;
           const uint32_t qpar = C::NDQ == 2 ? (((ng >> 1) & 1) ^ 1) : (uint32_t)((ng & 1) ^ 1);
           const bool more = n + 1 < w.n_steps;
-          if (!mbar_wait(bar(C::B_PT), ng & 1, abort_flag)) { ok = false; break; }
+          if (!pt_ready && !mbar_wait(bar(C::B_PT), ng & 1, abort_flag)) { ok = false; break; }
           if (n == 0 && in > 0 && !mbar_wait(bar(C::B_EPI), (in - 1) & 1, abort_flag)) { ok = false; break; }
+          const bool q_ready = !more || mbar_test(bar(C::B_QFULL + s1), ((ng + 1) / C::STAGES) & 1);
           tc_fence_after();
           issue_grad(C::T_ST, stage(do_mn, s), C::T_DV, n > 0);                 // dV += P^T dO
+          const bool ds_ready = mbar_test(bar(C::B_DS), ng & 1);
           if (more) {
-            if (!mbar_wait(bar(C::B_QFULL + s1), ((ng + 1) / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+            if (!q_ready && !mbar_wait(bar(C::B_QFULL + s1), ((ng + 1) / C::STAGES) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             issue_sdp(k_kmaj, stage(q_kmaj, s1), C::T_ST);                      // S^T for the next step
             mma_commit(bar(C::B_ST));
@@ -511,15 +521,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_commit(bar(C::B_DPT + db1));
             }
           }
-          if (!mbar_wait(bar(C::B_DS), ng & 1, abort_flag)) { ok = false; break; }
+          if (!ds_ready && !mbar_wait(bar(C::B_DS), ng & 1, abort_flag)) { ok = false; break; }
+          const bool dq_ready = mbar_test(bar(C::B_DQEMPTY + qslot), qpar);
           tc_fence_after();
           issue_grad(C::T_DPT + db * BM, stage(q_mn, s), C::T_DK, n > 0);       // dK += dS^T Q
           mma_commit(bar(C::B_QEMPTY + s));
-          if (!mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) { ok = false; break; }
+          if (!dq_ready && !mbar_wait(bar(C::B_DQEMPTY + qslot), qpar, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_dq(b2, C::T_DQ + qslot * C::DQ_COLS);                           // dQ_i partial
           mma_commit(bar(C::B_DQFULL + qslot));
           mma_commit(bar(C::B_DSFREE + b2));
+          pt_ready = more && mbar_test(bar(C::B_PT), (ng + 1) & 1);
           if (C::NDPT == 1 && more) {
             issue_dpt(stage(do_kmaj, s1), C::T_DPT);                            // dP^T for the next step
             mma_commit(bar(C::B_DPT));

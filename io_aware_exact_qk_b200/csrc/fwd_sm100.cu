@@ -366,15 +366,21 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           }
         if (!ok) break;
         mma_commit(bar(C::B_KEMPTY + s0));
+        // The V and K stages and the other tile's P are checked with mbar_test while the
+        // preceding MMAs issue (mbar_wait only if they had not completed then): a check that
+        // waits for its own shared-memory round trip leaves the tensor pipe's short queue idle.
+        bool v_ready = false;   // V tile of step j seen complete during step j - 1
         for (int j = 0; ok && j < it.nkv; ++j) {
           const uint32_t c = kv + j;
           const int s = c % C::STAGES;
-          if (!mbar_wait(bar(C::B_VFULL + s), (c / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+          if (!v_ready && !mbar_wait(bar(C::B_VFULL + s), (c / C::STAGES) & 1, abort_flag)) { ok = false; break; }
           bool k_next = false;
           const int s1 = (c + 1) % C::STAGES;
+          const bool k_ready = j + 1 < it.nkv && mbar_test(bar(C::B_KFULL + s1), ((c + 1) / C::STAGES) & 1);
+          bool p_ready = false;   // this tile's P seen complete while the other tile's products issued
           for (int t = 0; t < 2; ++t) {
             if (j >= it.n[t]) continue;
-            if (!mbar_wait(bar(C::B_PFULL + t), pc[t] & 1, abort_flag)) { ok = false; break; }
+            if (!p_ready && !mbar_wait(bar(C::B_PFULL + t), pc[t] & 1, abort_flag)) { ok = false; break; }
             ++pc[t];
             if (j == 0) {   // O_t of the previous item has been read out
               if (!mbar_wait(bar(C::B_OFREE + t), (om[t] & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -382,9 +388,13 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
             }
             tc_fence_after();
             issue_pv(t, s, j > 0);
+            p_ready = t == 0 && j < it.n[1] && mbar_test(bar(C::B_PFULL + 1), pc[1] & 1);
             if (j + 1 < it.n[t]) {
               if (!k_next) {
-                if (!mbar_wait(bar(C::B_KFULL + s1), ((c + 1) / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+                if (!k_ready && !mbar_wait(bar(C::B_KFULL + s1), ((c + 1) / C::STAGES) & 1, abort_flag)) {
+                  ok = false;
+                  break;
+                }
                 tc_fence_after();
                 k_next = true;
               }
@@ -396,6 +406,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
             }
           }
           if (!ok) break;
+          v_ready = j + 1 < it.nkv && mbar_test(bar(C::B_VFULL + s1), ((c + 1) / C::STAGES) & 1);
           mma_commit(bar(C::B_VEMPTY + s));
           if (k_next) mma_commit(bar(C::B_KEMPTY + s1));
         }

@@ -67,6 +67,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking check of the phase with the given parity (true: it has completed).  Its
+// result is used later than it is issued, so the shared-memory round trip overlaps the
+// instructions in between -- the MMA issuers start the check one MMA group ahead and fall
+// back to mbar_wait only when the phase had not completed yet.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  `abort_flag` (shared memory) is
 // set by whichever thread of the CTA first gives up; later waits then return at once.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
