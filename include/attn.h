@@ -105,6 +105,25 @@ attn_status attn_bwd(const void *q, const void *k, const void *v,
                      void *dq, void *dk, void *dv,
                      void *workspace, size_t workspace_bytes, void *stream);
 
+/* Backward into float32 accumulators: the gradients of the same backward (bf16 q, k, v,
+ * o, dout; float32 lse; same shape arguments and causal rule as attn_bwd) are ADDED to
+ *     dq_acc [T,hq,d],  dk_acc and dv_acc [T,hkv,d]      float32, DEVICE, 16-byte aligned
+ * (read-add-write; they must hold the running sums, zero before the first call) and nothing
+ * is written in bf16.  For computations that sum gradients over several calls -- ring
+ * attention's backward sums one call per K/V block it visits ("相关工作" page, paper 7) --
+ * this keeps the sum in float32 instead of rounding every call's gradients to bf16.  A
+ * call's contributions equal attn_bwd's before their bf16 rounding (dK, dQ include the
+ * scale).  Workspace: attn_bwd_workspace_size(..., ATTN_BF16).  Errors as attn_bwd; calls
+ * that add into the same accumulators must not overlap on the GPU. */
+attn_status attn_bwd_accumulate(const void *q, const void *k, const void *v,
+                                const void *o, const void *dout, const float *lse,
+                                const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
+                                int32_t max_seqlen, int32_t total_tokens,
+                                int32_t hq, int32_t hkv, int32_t d,
+                                float scale, int32_t causal,
+                                float *dq_acc, float *dk_acc, float *dv_acc,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
 /* Backward without a caller-provided workspace.  (The pages describe no counterpart; this
  * exists for callers that cannot allocate device memory where they run the backward:
  * engines that reserve all device memory up front and forbid allocation later, and plain

@@ -68,6 +68,9 @@ def load_library():
     lib.attn_profile_kernel_name.restype = ctypes.c_char_p
     lib.attn_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), i32]
     lib.attn_profile_collect.restype = ctypes.c_int
+    lib.attn_bwd_accumulate.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                        vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd_accumulate.restype = ctypes.c_int
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                      vp, vp, vp, vp]
     lib.attn_bwd_noalloc.restype = ctypes.c_int
@@ -182,6 +185,27 @@ def attn_bwd(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scale=None, 
                         ms, T, hq, hkv, d, float(scale), int(bool(causal)), _dtype_code(q), _ptr(dq), _ptr(dk),
                         _ptr(dv), _ptr(workspace), ws if workspace is not None else 0, _stream(stream)))
     return dq, dk, dv
+
+
+def attn_bwd_accumulate(q, k, v, o, do, lse, dq_acc, dk_acc, dv_acc, cu_seqlens=None, max_seqlen=None, scale=None,
+                        causal=False, batch=None, workspace=None, stream=None):
+    """Backward that ADDS its gradients into the float32 tensors dq_acc [T,Hq,d], dk_acc,
+    dv_acc [T,Hkv,d] (bf16 inputs); returns them."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (dq_acc, dk_acc, dv_acc):
+        if t.dtype != torch.float32:
+            raise AttnError(ATTN_ERR_INVALID_ARG, "the accumulators must be float32")
+    ws = workspace_size("bwd", q, k, cu_seqlens, max_seqlen, batch)
+    if ws and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _check(lib.attn_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(cu_seqlens), b,
+                                   seqlen, ms, T, hq, hkv, d, float(scale), int(bool(causal)), _ptr(dq_acc),
+                                   _ptr(dk_acc), _ptr(dv_acc), _ptr(workspace), ws if workspace is not None else 0,
+                                   _stream(stream)))
+    return dq_acc, dk_acc, dv_acc
 
 
 def attn_bwd_noalloc(q, k, v, o, do, lse, cu_seqlens=None, max_seqlen=None, scale=None, causal=False,

@@ -497,6 +497,26 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                    "attn_bwd (fp32 check mode) launch");
 }
 
+attn_status attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                const float* lse, const int32_t* cu_seqlens, int32_t batch, int32_t seqlen,
+                                int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d,
+                                float scale, int32_t causal, float* dq_acc, float* dk_acc, float* dv_acc,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  Problem pb;
+  attn_status st = (attn_status)bwd_check_args(q, k, v, o, dout, lse, cu_seqlens, batch, seqlen, max_seqlen,
+                                               total_tokens, hq, hkv, d, scale, causal, ATTN_BF16, dq_acc, dk_acc,
+                                               dv_acc, &pb);
+  if (st != ATTN_OK) return st;
+  if (total_tokens == 0 || batch == 0) return ok();
+  const size_t need = attn_bwd_workspace_size(batch, pb.max_seqlen, total_tokens, hq, hkv, d, ATTN_BF16);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if ((st = check_ptr(workspace, "workspace"))) return st;
+  return from_cuda(launch_bwd_bf16_accumulate(pb, q, k, v, o, dout, lse, dq_acc, dk_acc, dv_acc, workspace,
+                                              static_cast<cudaStream_t>(stream)),
+                   "attn_bwd_accumulate launch");
+}
+
 attn_status attn_get_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return from_cuda(e, "stream synchronize");

@@ -139,7 +139,8 @@ struct BwdCfg {
   static constexpr int B_EPI = B_VT + 1;             // dK, dV read out of TMEM
   static constexpr int B_IFULL = B_EPI + 1;          // kItemSlots: item index written
   static constexpr int B_IEMPTY = B_IFULL + kItemSlots;   // kItemSlots: read by every role
-  static constexpr int NBARS = B_IEMPTY + kItemSlots;
+  static constexpr int B_DRAIN = B_IEMPTY + kItemSlots;   // the MMA issuer's completion at exit
+  static constexpr int NBARS = B_DRAIN + 1;
   // after the barriers: TMEM address, abort flag, the item-index ring
   static constexpr int SMEM_BYTES = 1024 + O_BAR + NBARS * 8 + 8 + 4 * kItemSlots;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -166,6 +167,12 @@ struct BwdParams {
   float* dq_acc;         // [T, hq, d]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  // accumulate mode: dK and dV are added into these float32 [T, hkv, d] tensors (and dQ,
+  // scaled, into dq_acc, which is then the caller's) instead of being written as bf16
+  int32_t accumulate;
+  float dq_mul;          // factor on each dQ partial: scale in accumulate mode, else 1
+  float* dk_acc;
+  float* dv_acc;
 };
 
 // Enumerates the (query head, query tile) steps of one CTA in a fixed order.
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float nl[PER_LANE], nd[PER_LANE];
     int ng = 0;          // steps so far (all items)
     int in = 0;          // non-empty items so far
+    uint32_t kc = 0, qc = 0;   // K-buffer and Q / dO stage loads issued
     bool ok = true;
     for (int k = 0; ok; ++k) {
       // claim the next item and hand its index to the other roles
@@ -345,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pn * C::PANEL, w.g, w.seq_start + w.kv0);
         }
       }
+      ++kc;
       auto fetch = [&](int n) {
         int h, i;
         w.it.head_tile(n, w.g, &h, &i);
@@ -384,8 +393,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pn * C::PANEL, h, w.seq_start + q0);
           }
         }
+        ++qc;
       }
       ++in;
+    }
+    // Every load issued here lands before the CTA releases its memory, also when another
+    // role gave up waiting: only the last load of each buffer / stage can still be in flight.
+    if (lane == 0) {
+      for (uint32_t i = kc > (uint32_t)C::KV_BUFS ? kc - C::KV_BUFS : 0; i < kc; ++i)
+        mbar_wait_drain(bar(C::B_KFULL + i % C::KV_BUFS), (i / C::KV_BUFS) & 1);
+      for (uint32_t i = qc > (uint32_t)C::STAGES ? qc - C::STAGES : 0; i < qc; ++i)
+        mbar_wait_drain(bar(C::B_QFULL + i % C::STAGES), (i / C::STAGES) & 1);
     }
   } else if (warp == 13) {
     // ---------------- MMA issuer ----------------
@@ -541,6 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ng0 += w.n_steps;
         ++in;
       }
+      // every MMA issued here has completed before the CTA frees Tensor Memory
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait_drain(bar(C::B_DRAIN), 0);
     }
   } else if (warp < 8) {
     // ---------------- compute: P^T, dS^T for one key row and half of the query columns ----
@@ -687,7 +708,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------- epilogue: warps 0-3 write dV, warps 4-7 write dK = scale * acc ------
     if (!ok || !mbar_wait(bar(C::B_DONE), in & 1, abort_flag)) { ok = false; break; }
-    {
+    if (p.accumulate) {
+      tc_fence_after();
+      // float32 read-add-write of this thread's key row (each key row of the call belongs to
+      // exactly one item, so no other CTA touches it)
+      float* acc = half == 0 ? p.dv_acc : p.dk_acc;
+      const float mul = half == 0 ? 1.f : p.scale;
+      const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
+      const bool in_seq = kj < len;
+      float4* row = reinterpret_cast<float4*>(acc + ((size_t)(seq_start + (in_seq ? kj : 0)) * p.hkv + g) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(trow + col + c * 32, r);
+        tmem_wait_ld();
+        if (in_seq) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float4 a = row[c * 8 + e];
+            a.x += __uint_as_float(r[4 * e]) * mul;
+            a.y += __uint_as_float(r[4 * e + 1]) * mul;
+            a.z += __uint_as_float(r[4 * e + 2]) * mul;
+            a.w += __uint_as_float(r[4 * e + 3]) * mul;
+            row[c * 8 + e] = a;
+          }
+        }
+      }
+      const int kb = in % C::KV_BUFS;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(C::B_EPI));
+        mbar_arrive(bar(C::B_KEMPTY + kb));
+      }
+    } else {
       tc_fence_after();
       // Every product of the item has completed, so its K buffer is idle: each warp stages
       // its 32 rows there (half a row per pass at d = 128) and stores whole 128-byte row
@@ -794,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < C::STG_ROWS; ++e) {
             const int row = part * C::STG_ROWS + e;
-            stg[e * D + c] = __uint_as_float(r[row / 32][row % 32]);
+            stg[e * D + c] = __uint_as_float(r[row / 32][row % 32]) * p.dq_mul;
           }
           fence_proxy_async_smem();
           named_barrier_sync(1, 128);
@@ -817,8 +871,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int e = pn * 32 + j * 4;
-            *reinterpret_cast<uint4*>(stg + pn * C::STG_PANEL_BYTES + sw128_offset(qr, j)) =
-                make_uint4(r[e / 32][e % 32], r[e / 32][e % 32 + 1], r[e / 32][e % 32 + 2], r[e / 32][e % 32 + 3]);
+            const float m = p.dq_mul;
+            *reinterpret_cast<float4*>(stg + pn * C::STG_PANEL_BYTES + sw128_offset(qr, j)) =
+                make_float4(__uint_as_float(r[e / 32][e % 32]) * m, __uint_as_float(r[e / 32][e % 32 + 1]) * m,
+                            __uint_as_float(r[e / 32][e % 32 + 2]) * m, __uint_as_float(r[e / 32][e % 32 + 3]) * m);
           }
         fence_proxy_async_smem();
         named_barrier_sync(1, 128);
@@ -847,7 +903,8 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout, int64_t rows, int hq,
                                                       int total_tokens, float* __restrict__ dd,
-                                                      float* __restrict__ dq_acc, int* __restrict__ item_counter) {
+                                                      float* __restrict__ dq_acc, int zero_acc,
+                                                      int* __restrict__ item_counter) {
   constexpr int TPR = D / 8;   // threads per row
   if (blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;   // the main kernel's work-item counter
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -871,9 +928,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __res
         acc = fmaf(x.x, y.x, acc);
         acc = fmaf(x.y, y.y, acc);
       }
-      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (zero_acc) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -910,15 +969,23 @@ int sm_count() {
   return n;
 }
 
+// Accumulate mode (acc != nullptr): dq_acc, dk_acc, dv_acc are the caller's float32
+// tensors; the gradients are added into them and nothing is written as bf16.
+struct BwdAccum {
+  float* dq_acc;
+  float* dk_acc;
+  float* dv_acc;
+};
+
 template <int D>
 cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                         cudaStream_t stream) {
+                         const BwdAccum* acc, cudaStream_t stream) {
   using C = BwdCfg<D>;
   const size_t T = (size_t)pb.total_tokens;
   float* dd = static_cast<float*>(workspace);
   const size_t dbytes = ((size_t)pb.hq * T * sizeof(float) + 255) & ~(size_t)255;
-  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbytes);
+  float* dq_acc = acc ? acc->dq_acc : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbytes);
   int* item_counter = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + dbytes +
                                              T * (size_t)pb.hq * (size_t)D * sizeof(float));
   const int64_t rows = (int64_t)T * pb.hq;
@@ -928,7 +995,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
     LaunchScope scope(K_BWD_PREPROCESS, stream);
     bwd_preprocess<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                    static_cast<const __nv_bfloat16*>(dout), rows, pb.hq,
-                                                   pb.total_tokens, dd, dq_acc, item_counter);
+                                                   pb.total_tokens, dd, dq_acc, acc ? 0 : 1, item_counter);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -971,6 +1038,10 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
   p.dq_acc = dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.accumulate = acc ? 1 : 0;
+  p.dq_mul = acc ? pb.scale : 1.f;
+  p.dk_acc = acc ? acc->dk_acc : nullptr;
+  p.dv_acc = acc ? acc->dv_acc : nullptr;
   cudaError_t e = cudaFuncSetAttribute(bwd_bf16_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (shared memory allows no more) walking its item list
@@ -981,6 +1052,7 @@ cudaError_t launch_bwd_d(const Problem& pb, const void* q, const void* k, const 
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
+  if (acc) return cudaSuccess;   // the caller's accumulator stays float32
   const int64_t n8 = rows * D / 8;
   const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)sm_count() * 16);
   LaunchScope scope(K_BWD_DQ_CONVERT, stream);
@@ -1002,9 +1074,22 @@ cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, con
                             cudaStream_t stream) {
   if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
   switch (pb.d) {
-    case 32: return launch_bwd_d<32>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
-    case 64: return launch_bwd_d<64>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
-    case 128: return launch_bwd_d<128>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, stream);
+    case 32: return launch_bwd_d<32>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, nullptr, stream);
+    case 64: return launch_bwd_d<64>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, nullptr, stream);
+    case 128: return launch_bwd_d<128>(pb, q, k, v, o, dout, lse, dq, dk, dv, workspace, nullptr, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_bwd_bf16_accumulate(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
+                                       const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                                       float* dv_acc, void* workspace, cudaStream_t stream) {
+  if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
+  const BwdAccum acc{dq_acc, dk_acc, dv_acc};
+  switch (pb.d) {
+    case 32: return launch_bwd_d<32>(pb, q, k, v, o, dout, lse, nullptr, nullptr, nullptr, workspace, &acc, stream);
+    case 64: return launch_bwd_d<64>(pb, q, k, v, o, dout, lse, nullptr, nullptr, nullptr, workspace, &acc, stream);
+    case 128: return launch_bwd_d<128>(pb, q, k, v, o, dout, lse, nullptr, nullptr, nullptr, workspace, &acc, stream);
     default: return cudaErrorInvalidValue;
   }
 }

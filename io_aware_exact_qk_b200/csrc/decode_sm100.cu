@@ -65,7 +65,8 @@ struct DecCfg {
   static constexpr int B_SFULL = B_VEMPTY + STAGES;  // 2 (one per S buffer)
   static constexpr int B_PFULL = B_SFULL + 2;        // arrived once per active softmax warp
   static constexpr int B_PVDONE = B_PFULL + 1;       // committed after every PV
-  static constexpr int NBARS = B_PVDONE + 1;
+  static constexpr int B_DRAIN = B_PVDONE + 1;       // the MMA issuer's completion at exit
+  static constexpr int NBARS = B_DRAIN + 1;
   static constexpr int DATA_BYTES = (1 + 2 * STAGES) * TILE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + NBARS * 8 + 16;
 };
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar(C::B_QFULL), (uint32_t)(D * 2 * p.G * p.max_seqlen_q));
       for (int pn = 0; pn < C::NPANEL; ++pn)
         tma_load_3d(sQ + pn * C::PANEL_BYTES, &tmQ, bar(C::B_QFULL), pn * C::PANEL, g * p.G, q0);
+      int kc = 0, vc = 0;   // K and V loads issued
       for (int i = 0; i < n; ++i) {
         const int s = i % C::STAGES;
         const uint32_t ph = (i / C::STAGES) & 1;
@@ -169,11 +171,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
         for (int pn = 0; pn < C::NPANEL; ++pn)
           tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, g, key);
+        ++kc;
         if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
         for (int pn = 0; pn < C::NPANEL; ++pn)
           tma_load_3d(sV + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, bar(C::B_VFULL + s), pn * C::PANEL, g, key);
+        ++vc;
       }
+      // Every load issued here lands before the CTA releases its memory, also when another
+      // role gave up waiting: only the last load of each stage can still be in flight.
+      mbar_wait_drain(bar(C::B_QFULL), 0);
+      for (int i = kc > C::STAGES ? kc - C::STAGES : 0; i < kc; ++i)
+        mbar_wait_drain(bar(C::B_KFULL + i % C::STAGES), (i / C::STAGES) & 1);
+      for (int i = vc > C::STAGES ? vc - C::STAGES : 0; i < vc; ++i)
+        mbar_wait_drain(bar(C::B_VFULL + i % C::STAGES), (i / C::STAGES) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer: S(0), S(1), then PV(i), S(i+2) ----------------
@@ -213,6 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(C::B_PVDONE));
         if (i + 2 < n) ok = issue_s(i + 2);
       }
+      // every MMA issued here has completed before the CTA frees Tensor Memory
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait_drain(bar(C::B_DRAIN), 0);
     }
   } else if (warp < n_active) {
     // ---------------- softmax + epilogue, one packed query row per thread ----------------

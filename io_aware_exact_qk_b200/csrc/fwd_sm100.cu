@@ -95,7 +95,8 @@ struct FwdCfg {
   static constexpr int B_OFREE = B_OFINAL + 2;       // 2
   static constexpr int B_IFULL = B_OFREE + 2;        // kItemSlots: item index written
   static constexpr int B_IEMPTY = B_IFULL + kItemSlots;   // kItemSlots: read by MMA + softmax warps
-  static constexpr int NBARS = B_IEMPTY + kItemSlots;
+  static constexpr int B_DRAIN = B_IEMPTY + kItemSlots;   // the MMA issuer's completion at exit
+  static constexpr int NBARS = B_DRAIN + 1;
   // Epilogue staging: each softmax warp turns its 32 O rows into coalesced stores through a
   // 32-row slice of STG_ROWB bytes per row (half a row per pass at d = 128).
   static constexpr int STG_ROWB = D * 2 < 128 ? D * 2 : 128;
@@ -253,6 +254,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
     if (lane == 0) {
       uint32_t kv = 0;            // K/V tiles so far
       uint32_t qc[2] = {0, 0};    // loads of each query tile buffer so far
+      uint32_t kc = 0, vc = 0;    // K and V loads issued
       bool ok = true;
       for (int k = 0; ok; ++k) {
         // claim the next item and hand its index to the other roles
@@ -288,9 +290,11 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           for (int pn = 0; pn < C::NPANEL; ++pn)
             tma_load_3d(sK + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, bar(C::B_KFULL + s), pn * C::PANEL, hk,
                         it.seq_start + j * kKeys);
+          ++kc;
           if (j == 0 && !load_q(1)) { ok = false; break; }
           if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
+          ++vc;
           if constexpr (FP8) {
             // V^T [batch * hkv][d][padded seqlen]: a (128 keys) x (d rows) box, keys
             // contiguous (K-major B); the key coordinate is a multiple of 128
@@ -302,6 +306,15 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
           }
         }
       }
+      // Every load issued here lands before the CTA releases its memory, also when another
+      // role gave up waiting: only the last load of each stage can still be in flight (a
+      // stage is reloaded only after its previous contents were consumed).
+      for (uint32_t i = kc > (uint32_t)C::STAGES ? kc - C::STAGES : 0; i < kc; ++i)
+        mbar_wait_drain(bar(C::B_KFULL + i % C::STAGES), (i / C::STAGES) & 1);
+      for (uint32_t i = vc > (uint32_t)C::STAGES ? vc - C::STAGES : 0; i < vc; ++i)
+        mbar_wait_drain(bar(C::B_VFULL + i % C::STAGES), (i / C::STAGES) & 1);
+      for (int t = 0; t < 2; ++t)
+        if (qc[t] > 0) mbar_wait_drain(bar(C::B_QFULL + t), (qc[t] - 1) & 1);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
@@ -412,6 +425,9 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap& tmQ, const CUtensorM
         }
         kv += it.nkv;
       }
+      // every MMA issued here has completed before the CTA frees Tensor Memory
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait_drain(bar(C::B_DRAIN), 0);
     }
   } else {
     // ---------------- softmax / correction / epilogue (one query row per thread) ---------

@@ -31,6 +31,13 @@ cudaError_t launch_bwd_bf16(const Problem& pb, const void* q, const void* k, con
                             const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
                             cudaStream_t stream);
 
+// The same backward adding its gradients into the caller's float32 dq_acc [T,hq,d],
+// dk_acc and dv_acc [T,hkv,d] (read-add-write; nothing bf16 is written).  Workspace:
+// bwd_bf16_workspace_bytes(pb) (its dQ accumulator part goes unused).
+cudaError_t launch_bwd_bf16_accumulate(const Problem& pb, const void* q, const void* k, const void* v, const void* o,
+                                       const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                                       float* dv_acc, void* workspace, cudaStream_t stream);
+
 // Decoding-shaped forward (split-KV): sequence b has Lq query rows (the newest positions)
 // and Lk keys.  q [Tq,hq,d], k/v [Tk,hkv,d], o [Tq,hq,d] bf16, lse [hq,Tq] f32.
 struct DecodeProblem {

@@ -101,6 +101,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait used when a role drains its own asynchronous work at the end of a kernel:
+// unlike mbar_wait it does not give up when another role has aborted, since the CTA must
+// not free its shared memory or Tensor Memory while its own copies or MMAs are in flight.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 255u) == 0u && globaltimer_ns() - t0 > *(volatile uint64_t*)&g_wait_limit_ns) {
+      report_error(ATTN_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ---- TMA ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

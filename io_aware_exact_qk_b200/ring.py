@@ -20,14 +20,16 @@ The backward walks the same ring.  With the full forward's O and LSE of this ran
 of the (query chunk, K/V block) pair given those O and LSE (the tutorial's 反向重算流程:
 P is recomputed from the saved LSE, D from the saved O), so dQ is the sum of the per-hop
 dQ, and each block's dK / dV accumulate as the block travels: they are passed on with it
-after every hop and arrive back at the block's owner after the last one.
+after every hop and arrive back at the block's owner after the last one.  The sums are
+float32 throughout: every hop's backward adds straight into them (attn_bwd_accumulate),
+and they are rounded to bf16 once, at the end.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
-from . import attn_bwd, attn_fwd, attn_merge_finish, attn_merge_partial
+from . import attn_bwd_accumulate, attn_fwd, attn_merge_finish, attn_merge_partial
 
 
 def ring_schedule(rank: int, world: int, causal: bool):
@@ -90,19 +92,22 @@ def ring_attn_fwd(q, k, v, batch, scale=None, causal=False, group=None, local_fw
     return finish(o_acc), lse_acc
 
 
-def ring_attn_bwd(q, k, v, o, do, lse, batch, scale=None, causal=False, group=None, local_bwd=None,
+def ring_attn_bwd(q, k, v, o, do, lse, batch, scale=None, causal=False, group=None, local_bwd=None, finish=None,
                   acc_dtype=torch.float32):
     """Gradients of the ring forward for this rank: (dq [B n, Hq, d] for its query chunk,
-    dk, dv [B n, Hkv, d] for its K/V chunk), in the dtypes of q, k, v.  ``o`` / ``lse`` are
-    this rank's rows of the full forward (``ring_attn_fwd``'s outputs), ``do`` their
-    upstream gradient.  ``local_bwd(q, k, v, causal) -> (dq, dk, dv)`` defaults to the
-    library's attn_bwd on the pair with the given o, do, lse; partial gradients are summed
-    in ``acc_dtype``."""
+    dk, dv [B n, Hkv, d] for its K/V chunk).  ``o`` / ``lse`` are this rank's rows of the
+    full forward (``ring_attn_fwd``'s outputs), ``do`` their upstream gradient.
+    ``local_bwd(q, k, v, causal, dq_acc, dk_acc, dv_acc)`` adds the pair's gradients into the
+    ``acc_dtype`` accumulators; it defaults to the library's attn_bwd_accumulate with the given
+    o, do, lse.  ``finish(acc) -> tensor`` turns an accumulator into the result; by default
+    the library's attn_merge_finish (float32 to bf16)."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     if local_bwd is None:
-        def local_bwd(q_, k_, v_, c_):
-            return attn_bwd(q_, k_, v_, o, do, lse, scale=scale, causal=c_, batch=batch)
+        def local_bwd(q_, k_, v_, c_, dq_a, dk_a, dv_a):
+            attn_bwd_accumulate(q_, k_, v_, o, do, lse, dq_a, dk_a, dv_a, scale=scale, causal=c_, batch=batch)
+    if finish is None:
+        finish = attn_merge_finish
     nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
     prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
     dq_acc = torch.zeros(q.shape, dtype=acc_dtype, device=q.device)
@@ -118,10 +123,7 @@ def ring_attn_bwd(q, k, v, o, do, lse, batch, scale=None, causal=False, group=No
                 dist.P2POp(dist.isend, k_cur, nxt, group), dist.P2POp(dist.irecv, k_nxt, prv, group),
                 dist.P2POp(dist.isend, v_cur, nxt, group), dist.P2POp(dist.irecv, v_nxt, prv, group)])
         if kind is not None:
-            dq_p, dk_p, dv_p = local_bwd(q, k_cur, v_cur, kind == "causal")
-            dq_acc += dq_p.to(acc_dtype)
-            dk_cur += dk_p.to(acc_dtype)
-            dv_cur += dv_p.to(acc_dtype)
+            local_bwd(q, k_cur, v_cur, kind == "causal", dq_acc, dk_cur, dv_cur)
         # the block's gradients so far go on with it (after the last hop: to its owner)
         g_reqs = []
         if world > 1:
@@ -135,4 +137,4 @@ def ring_attn_bwd(q, k, v, o, do, lse, batch, scale=None, causal=False, group=No
             dk_cur, dv_cur = dk_in, dv_in
         if s + 1 < world:
             k_cur, v_cur = k_nxt, v_nxt
-    return dq_acc.to(q.dtype), dk_cur.to(k.dtype), dv_cur.to(v.dtype)
+    return finish(dq_acc), finish(dk_cur), finish(dv_cur)

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 import attn_workloads as W
+import io_aware_exact_qk_b200 as attn
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu
@@ -75,3 +76,29 @@ def test_fp32_check_mode(d, causal):
         g = P.to_np(g)
         assert P.rel_l2(g, r) <= P.FP32_REL, name
         assert P.max_rel(g, r) <= P.FP32_REL, name
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_accumulate_mode_adds_float32_gradients(d, causal):
+    """attn_bwd_accumulate adds the gradients into float32 tensors: two calls on the same
+    inputs give twice the gradient (each call within the backward's tolerance of the
+    oracle), and one call agrees with attn_bwd up to attn_bwd's own bf16 rounding."""
+    w = W.custom(f"acc_d{d}", [1, 130, 0, 257], 8, 2, d, causal, seed=90 + d)
+    q, k, v, do, cu = W.make_inputs(w)
+    qd, kd, vd, dod, cud = (t.cuda() for t in (q, k, v, do, cu))
+    kw = dict(cu_seqlens=cud, max_seqlen=w.max_seqlen, scale=w.scale, causal=causal)
+    o, lse = attn.attn_fwd(qd, kd, vd, **kw)
+    accs = [torch.zeros(t.shape, dtype=torch.float32, device="cuda") for t in (qd, kd, vd)]
+    attn.attn_bwd_accumulate(qd, kd, vd, o, dod, lse, *accs, **kw)
+    once = [P.to_np(a) for a in accs]
+    attn.attn_bwd_accumulate(qd, kd, vd, o, dod, lse, *accs, **kw)
+    attn.attn_get_device_error()
+    twice = [P.to_np(a) for a in accs]
+    ref = P.oracle_bwd(w, q, k, v, do, cu)[:3]
+    P.check_grads_bf16(once, ref, tag=w.name)
+    for a, b in zip(once, twice):
+        assert P.rel_l2(b, 2 * a) <= 1e-6
+    bf = [P.to_np(t) for t in attn.attn_bwd(qd, kd, vd, o, dod, lse, **kw)]
+    for name, a, b in zip(("dq", "dk", "dv"), once, bf):
+        assert np.abs(a - b).max() <= 2 ** -8 * np.abs(a).max() + 1e-6, name

@@ -67,10 +67,11 @@ def test_emulated_ring_matches_full_attention(world, causal, d):
 
 @pytest.mark.parametrize("world,causal,d", [(2, True, 128), (3, False, 64), (4, True, 32)])
 def test_emulated_ring_backward_matches_the_gradient(world, causal, d):
-    """Every rank's hops run attn_bwd on its (query chunk, K/V block) pairs with its rows of
-    the full forward's O and LSE; dQ sums over the rank's hops, dK / dV of a block over the
-    ranks it visits.  The stored O (bf16) and LSE (fp32) are the oracle's forward, given to
-    the oracle's backward as well (the backward as a function of its inputs)."""
+    """Every rank's hops run attn_bwd_accumulate on its (query chunk, K/V block) pairs with
+    its rows of the full forward's O and LSE, adding into float32 sums: dQ over the rank's
+    hops, dK / dV of a block over the ranks it visits (as ring_attn_bwd does).  The stored O
+    (bf16) and LSE (fp32) are the oracle's forward, given to the oracle's backward as well
+    (the backward as a function of its inputs)."""
     batch, n, hq, hkv = 2, 256 if d == 128 else 200, 8, 2
     N = world * n
     w = W.custom("ring-bwd", [N] * batch, hq, hkv, d, causal, 3300 + world)
@@ -88,11 +89,8 @@ def test_emulated_ring_backward_matches_the_gradient(world, causal, d):
         for j, kind in ring_schedule(r, world, causal):
             if kind is None:
                 continue
-            gq, gk, gv = attn.attn_bwd(qs[r], ks[j], vs[j], os_[r], dos[r], lses[r], scale=w.scale,
-                                       causal=kind == "causal", batch=batch)
-            dq[r] += gq.float()
-            dk[j] += gk.float()
-            dv[j] += gv.float()
+            attn.attn_bwd_accumulate(qs[r], ks[j], vs[j], os_[r], dos[r], lses[r], dq[r], dk[j], dv[j],
+                                     scale=w.scale, causal=kind == "causal", batch=batch)
     attn.attn_get_device_error()
     dq_r, dk_r, dv_r, _, _ = oracle.attn_bwd(q, k, v, do, cu.numpy(), scale=w.scale, causal=causal,
                                              o=o_st.double().numpy(), lse=lse_st.double().numpy())

@@ -51,12 +51,13 @@ def _merge64(o_acc, lse_acc, o_p, lse_p, first):
 
 
 def _local_oracle_bwd(batch, scale, o, do, lse):
-    def f(q, k, v, causal):
+    def f(q, k, v, causal, dq_acc, dk_acc, dv_acc):
         n = q.shape[0] // batch
         cu = np.arange(batch + 1, dtype=np.int32) * n
         dq, dk, dv, _, _ = oracle.attn_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), cu, scale=scale,
                                            causal=causal, threads=1, o=o.numpy(), lse=lse.numpy())
-        return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+        for acc, g in ((dq_acc, dq), (dk_acc, dk), (dv_acc, dv)):
+            acc.add_(torch.from_numpy(g))
     return f
 
 
@@ -80,7 +81,8 @@ def _worker(rank, world, port, batch, n, hq, hkv, d, causal, out):
         o, lse = ring_attn_fwd(qc, kc, vc, batch, scale=scale, causal=causal, local_fwd=_local_oracle(batch, scale),
                                merge=_merge64, finish=lambda oa: oa, acc_dtype=torch.float64)
         dq, dk, dv = ring_attn_bwd(qc, kc, vc, o, doc, lse, batch, scale=scale, causal=causal,
-                                   local_bwd=_local_oracle_bwd(batch, scale, o, doc, lse), acc_dtype=torch.float64)
+                                   local_bwd=_local_oracle_bwd(batch, scale, o, doc, lse), finish=lambda a: a,
+                                   acc_dtype=torch.float64)
         out[rank] = (o.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy())
         dist.barrier()
     finally:
