@@ -43,8 +43,9 @@
 // dQ_i = dS K_j (M = 128 query rows, N = d): 128 + 128 + 4 d <= 512 columns.
 //
 // Warp roles (448 threads): two compute warpgroups, each owning half of the query columns
-// of every step (P^T, dS^T) and one of the dK / dV epilogues (which also load the next
-// item's V_j into TMEM); a dQ drain warpgroup; a TMA producer warp that claims the items
+// of every step (P^T, dS^T) and one of the dK / dV epilogues; a dQ drain warpgroup (which
+// also loads each item's V_j into TMEM, during the previous item's epilogue); a TMA
+// producer warp that claims the items
 // (+ LSE / D rows into SMEM, one step ahead); an MMA issuer warp.  Across items the
 // pipelines keep running: the next item's K_j and first Q / dO tiles load during the
 // current item, and its first products start while the epilogue drains dK / dV.
@@ -237,7 +238,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
 // Warp roles (448 threads):
 //   warps 0-3   compute, query columns [0, BM/2) of every step, then the dV epilogue
 //   warps 4-7   compute, query columns [BM/2, BM), then the dK epilogue
-//   warps 8-11  dQ drain
+//   warps 8-11  dQ drain; also loads each item's V_j into TMEM
 //   warp  12    producer (TMA for K, V, Q_i, dO_i; LSE_i, D_i rows into SMEM)
 //   warp  13    MMA issuer
 template <int D>
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
       // warp-level arrivals: one per compute warp (PT, DS, K buffer free, epilogue read
-      // out) or drain warp (DQEMPTY), one per first-warpgroup warp for V in TMEM
+      // out) or drain warp (DQEMPTY, V in TMEM)
       if (i == C::B_PT || i == C::B_DS || i == C::B_EPI || i == C::B_KEMPTY || i == C::B_KEMPTY + 1) cnt = 8;
       if (i == C::B_DQEMPTY || i == C::B_DQEMPTY + 1 || i == C::B_VT) cnt = 4;
       // item slots are read by the MMA warp, the 8 compute warps and the 4 drain warps
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           issue_sdp(k_kmaj, stage(q_kmaj, s0), C::T_ST);
           mma_commit(bar(C::B_ST));
-          // V_j of this item in TMEM (its compute warps load it after the previous item)
+          // V_j of this item in TMEM (the drain loads it once the previous item's dP^T are done)
           ok = !C::VT || mbar_wait(bar(C::B_VT), in & 1, abort_flag);
         }
         if (ok) {
@@ -581,42 +582,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (w.n_steps == 0) continue;
     const int g = w.g, seq_start = w.seq_start, len = w.len, kv0 = w.kv0;
     const int kj = kv0 + kr;                      // key index inside the sequence
-    if (C::VT && half == 0) {
-      // V_j row kr, bf16 pairs as they lie in memory (element 2c in the low half of column
-      // c), is the A operand of dP^T; rows past the sequence are zero.  (The previous
-      // item's products are all done: its epilogue waited for them.)
-      const uint4* vrow = reinterpret_cast<const uint4*>(p.v + ((size_t)(seq_start + kj) * p.hkv + g) * D);
-      if constexpr (C::V_COLS >= 32) {
-#pragma unroll
-        for (int cb = 0; cb < C::V_COLS; cb += 32) {
-          uint32_t w[32];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint4 x = kj < len ? vrow[cb / 4 + e] : make_uint4(0u, 0u, 0u, 0u);
-            w[4 * e] = x.x;
-            w[4 * e + 1] = x.y;
-            w[4 * e + 2] = x.z;
-            w[4 * e + 3] = x.w;
-          }
-          tmem_st32(trow + C::T_V + cb, w);
-        }
-      } else {   // d = 32: a 64-byte row, 16 columns
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint4 x = kj < len ? vrow[e] : make_uint4(0u, 0u, 0u, 0u);
-          w[4 * e] = x.x;
-          w[4 * e + 1] = x.y;
-          w[4 * e + 2] = x.z;
-          w[4 * e + 3] = x.w;
-        }
-        tmem_st16(trow + C::T_V, w);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_VT));
-    }
     for (int n = 0; n < w.n_steps; ++n) {
       const int ng = ng0 + n;
       const int ls = ng % C::LSLOTS;
@@ -818,6 +783,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (idx < 0 || idx >= p.n_items) break;
     const BItem w = bitem_from<BM>(p, idx);
     const int seq_start = w.seq_start;
+    if (C::VT && w.n_steps > 0) {
+      // V_j into TMEM, row kr = this thread's lane: bf16 pairs as they lie in memory
+      // (element 2c in the low half of column c) form the A operand of dP^T; rows past the
+      // sequence are zero.  The drain does it (not the compute warps, which are writing the
+      // previous item's dK / dV out by now): V's columns are free once it has read the
+      // previous item's last dQ partial, whose completion follows every dP^T of that item.
+      const int kj = w.kv0 + lane_base + lane;
+      const uint4* vrow = reinterpret_cast<const uint4*>(p.v + ((size_t)(seq_start + kj) * p.hkv + w.g) * D);
+      if constexpr (C::V_COLS >= 32) {
+#pragma unroll
+        for (int cb = 0; cb < C::V_COLS; cb += 32) {
+          uint32_t vw[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint4 x = kj < w.len ? vrow[cb / 4 + e] : make_uint4(0u, 0u, 0u, 0u);
+            vw[4 * e] = x.x;
+            vw[4 * e + 1] = x.y;
+            vw[4 * e + 2] = x.z;
+            vw[4 * e + 3] = x.w;
+          }
+          tmem_st32(trow + C::T_V + cb, vw);
+        }
+      } else {   // d = 32: a 64-byte row, 16 columns
+        uint32_t vw[16];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint4 x = kj < w.len ? vrow[e] : make_uint4(0u, 0u, 0u, 0u);
+          vw[4 * e] = x.x;
+          vw[4 * e + 1] = x.y;
+          vw[4 * e + 2] = x.z;
+          vw[4 * e + 3] = x.w;
+        }
+        tmem_st16(trow + C::T_V, vw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_VT));
+    }
     for (int n = 0; n < w.n_steps; ++n, ++ng) {
       const int b2 = C::NDQ == 2 ? (ng & 1) : 0;                   // dQ slot
       const uint32_t par = C::NDQ == 2 ? ((ng >> 1) & 1) : (uint32_t)(ng & 1);
