@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ++in;
     }
   } else if (warp < 12) {
-    // ---------------- dQ drain: TMEM partial -> fp32 atomics into the accumulator ---------
+    // ---------------- dQ drain: TMEM partial -> staging tile -> bulk reduction into the accumulator
     const int lane_base = (warp & 3) * 32;
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     int ng = 0;          // steps so far (all items)
