@@ -203,7 +203,7 @@ attn_status attn_merge_finish(const float *o_acc, void *o, int32_t total_tokens,
  * (FlashAttention-3 on H100, 观察 2) and quantised attention with scaling (设计空间, 路线 4);
  * the scaling chosen here is one factor per head and tensor.
  * Reads bf16 q [batch*seqlen, hq, d], k and v [batch*seqlen, hkv, d] (a fixed-length
- * batch; d = 64 or 128) and writes, all on the device, caller-allocated, 16-byte aligned:
+ * batch; d = 64 or 128; attn_fp8_quantize_varlen below takes packed sequences) and writes, all on the device, caller-allocated, 16-byte aligned:
  *   descale_q [hq], descale_k [hkv], descale_v [hkv] float32: amax over the head / 448
  *       (1 for an all-zero head), 448 being the largest finite e4m3 value;
  *   q8 [batch*seqlen, hq, d], k8 [batch*seqlen, hkv, d] bytes: e4m3 of x / descale
@@ -234,6 +234,30 @@ attn_status attn_fwd_fp8(const void *q8, const void *k8, const void *vt8,
                          int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d,
                          float scale, int32_t causal, void *o, float *lse,
                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* The two FP8 calls over packed sequences of different lengths (the variable-length layout
+ * of attn_fwd): sequence b holds tokens cu_seqlens[b] .. cu_seqlens[b+1] - 1 of q, k, v, q8,
+ * k8, o (cu_seqlens: batch + 1 int32 on the device, non-decreasing, cu_seqlens[0] = 0,
+ * cu_seqlens[batch] = total_tokens; no sequence longer than max_seqlen).  V^T is
+ * vt8 [batch*hkv][d][pitch] with pitch = max_seqlen rounded up to a multiple of 16, sequence
+ * b's tokens in columns 0 .. len_b - 1 and zeros after them; the descales are per head over
+ * all sequences, as in the fixed-length calls.  attn_fwd_fp8_varlen reads what
+ * attn_fp8_quantize_varlen wrote with the same cu_seqlens and max_seqlen.  A sequence
+ * longer than max_seqlen is reported by attn_get_device_error (ATTN_ERR_INVALID_ARG); its
+ * V^T is cut at the pitch.  Errors: as the fixed-length calls, and ATTN_ERR_INVALID_ARG for
+ * a NULL cu_seqlens or max_seqlen > total_tokens. */
+attn_status attn_fp8_quantize_varlen(const void *q, const void *k, const void *v,
+                                     const int32_t *cu_seqlens, int32_t batch, int32_t max_seqlen,
+                                     int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d,
+                                     void *q8, void *k8, void *vt8,
+                                     float *descale_q, float *descale_k, float *descale_v,
+                                     void *stream);
+attn_status attn_fwd_fp8_varlen(const void *q8, const void *k8, const void *vt8,
+                                const float *descale_q, const float *descale_k,
+                                const float *descale_v, const int32_t *cu_seqlens, int32_t batch,
+                                int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
+                                int32_t d, float scale, int32_t causal, void *o, float *lse,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /* Workspace bytes attn_fwd / attn_bwd need for these shape arguments (0 = none). */
 size_t attn_fwd_workspace_size(int32_t batch, int32_t max_seqlen, int32_t total_tokens,

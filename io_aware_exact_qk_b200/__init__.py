@@ -86,6 +86,10 @@ def load_library():
     lib.attn_fp8_quantize.restype = ctypes.c_int
     lib.attn_fwd_fp8.argtypes = [vp] * 6 + [i32] * 5 + [f32, i32, vp, vp, vp, sz, vp]
     lib.attn_fwd_fp8.restype = ctypes.c_int
+    lib.attn_fp8_quantize_varlen.argtypes = [vp, vp, vp, vp] + [i32] * 6 + [vp] * 6 + [vp]
+    lib.attn_fp8_quantize_varlen.restype = ctypes.c_int
+    lib.attn_fwd_fp8_varlen.argtypes = [vp] * 7 + [i32] * 6 + [f32, i32, vp, vp, vp, sz, vp]
+    lib.attn_fwd_fp8_varlen.restype = ctypes.c_int
     lib.attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.attn_set_wait_limit_ns.restype = ctypes.c_int
     lib.attn_get_wait_limit_ns.argtypes = []
@@ -294,47 +298,54 @@ def attn_merge_finish(o_acc, o=None, stream=None):
 
 
 def fp8_vt_pitch(seqlen):
-    """Token pitch of the transposed e4m3 V: seqlen rounded up to a multiple of 16."""
+    """Token pitch of the transposed e4m3 V: the longest sequence rounded up to a multiple
+    of 16."""
     return (int(seqlen) + 15) // 16 * 16
 
 
-def attn_fp8_quantize(q, k, v, batch, stream=None):
-    """Per-head e4m3 operands of the FP8 forward from bf16 q [B S, Hq, 128], k, v
-    [B S, Hkv, 128]: returns (q8, k8 as uint8 [B S, H, 128], vt8 uint8 [B Hkv, 128, pitch],
-    descale_q [Hq], descale_k [Hkv], descale_v [Hkv] float32)."""
-    T, hq, d = q.shape
-    hkv = k.shape[1]
-    seqlen = T // batch if batch else 0
+def attn_fp8_quantize(q, k, v, batch=None, cu_seqlens=None, max_seqlen=None, stream=None):
+    """Per-head e4m3 operands of the FP8 forward from bf16 q [T, Hq, d], k, v [T, Hkv, d]
+    (d = 64 or 128; `batch` sequences of T / batch tokens, or the packed sequences of
+    cu_seqlens with max_seqlen): returns (q8, k8 as uint8 [T, H, d], vt8 uint8
+    [batch Hkv, d, fp8_vt_pitch(max_seqlen)], descale_q [Hq], descale_k [Hkv],
+    descale_v [Hkv] float32)."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
     dev = q.device
     q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
     k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
-    vt8 = torch.empty(batch * hkv, d, fp8_vt_pitch(seqlen), dtype=torch.uint8, device=dev)
+    vt8 = torch.empty(b * hkv, d, fp8_vt_pitch(ms), dtype=torch.uint8, device=dev)
     ds = [torch.empty(n, dtype=torch.float32, device=dev) for n in (hq, hkv, hkv)]
-    _check(load_library().attn_fp8_quantize(_ptr(q), _ptr(k), _ptr(v), batch, seqlen, hq, hkv, d, _ptr(q8), _ptr(k8),
-                                            _ptr(vt8), _ptr(ds[0]), _ptr(ds[1]), _ptr(ds[2]), _stream(stream)))
+    outs = (_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(ds[0]), _ptr(ds[1]), _ptr(ds[2]), _stream(stream))
+    if cu_seqlens is None:
+        _check(lib.attn_fp8_quantize(_ptr(q), _ptr(k), _ptr(v), b, seqlen, hq, hkv, d, *outs))
+    else:
+        _check(lib.attn_fp8_quantize_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), b, ms, T, hq, hkv, d, *outs))
     return q8, k8, vt8, ds[0], ds[1], ds[2]
 
 
-def attn_fwd_fp8(q8, k8, vt8, descale_q, descale_k, descale_v, batch, scale=None, causal=False, o=None, lse=None,
-                 workspace=None, stream=None):
-    """FP8 forward on attn_fp8_quantize's operands.  Returns (o [B S, Hq, 128] bf16,
-    lse [Hq, B S] fp32)."""
-    T, hq, d = q8.shape
-    hkv = k8.shape[1]
-    seqlen = T // batch if batch else 0
+def attn_fwd_fp8(q8, k8, vt8, descale_q, descale_k, descale_v, batch=None, scale=None, causal=False, o=None, lse=None,
+                 workspace=None, stream=None, cu_seqlens=None, max_seqlen=None):
+    """FP8 forward on attn_fp8_quantize's operands (the same batch, or the same cu_seqlens
+    and max_seqlen).  Returns (o [T, Hq, d] bf16, lse [Hq, T] fp32)."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q8, k8, cu_seqlens, max_seqlen, batch)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if o is None:
         o = torch.empty(T, hq, d, dtype=torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty(hq, T, dtype=torch.float32, device=q8.device)
-    ws = int(load_library().attn_fwd_workspace_size(batch, seqlen, T, hq, hkv, d, 0))
+    ws = int(lib.attn_fwd_workspace_size(b, ms, T, hq, hkv, d, 0))
     if ws and workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=q8.device)
-    _check(load_library().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(descale_q), _ptr(descale_k),
-                                       _ptr(descale_v), batch, seqlen, hq, hkv, d, float(scale), int(bool(causal)),
-                                       _ptr(o), _ptr(lse), _ptr(workspace), ws if workspace is not None else 0,
-                                       _stream(stream)))
+    operands = (_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v))
+    tail = (float(scale), int(bool(causal)), _ptr(o), _ptr(lse), _ptr(workspace),
+            ws if workspace is not None else 0, _stream(stream))
+    if cu_seqlens is None:
+        _check(lib.attn_fwd_fp8(*operands, b, seqlen, hq, hkv, d, *tail))
+    else:
+        _check(lib.attn_fwd_fp8_varlen(*operands, _ptr(cu_seqlens), b, ms, T, hq, hkv, d, *tail))
     return o, lse
 
 

@@ -221,16 +221,23 @@ bool encode_tma_3d_f32(void* tmap_out, const void* base, int d, int heads, int r
 using namespace attn;
 
 namespace {
-// Shapes of the FP8 calls: a fixed-length batch (batch sequences of seqlen tokens), d = 128.
-attn_status check_fp8(int32_t batch, int32_t seqlen, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+// Shapes of the FP8 calls: a fixed-length batch (cu_seqlens NULL: batch sequences of seqlen
+// tokens) or packed sequences (cu_seqlens, max_seqlen, total_tokens); d = 64 or 128.
+attn_status check_fp8(const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen,
+                      int32_t total_tokens, int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
                       Problem* pb) {
   if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 forward needs head dim 64 or 128 (got %d)", d);
-  if (batch < 0 || seqlen < 0) return fail(ATTN_ERR_INVALID_ARG, "negative batch / seqlen");
-  if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
+  if (batch < 0 || seqlen < 0 || max_seqlen < 0 || total_tokens < 0)
+    return fail(ATTN_ERR_INVALID_ARG, "negative batch / seqlen / max_seqlen / total_tokens");
+  if (cu_seqlens == nullptr) {
+    if ((int64_t)batch * seqlen > INT32_MAX) return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
+    max_seqlen = seqlen;
+    total_tokens = batch * seqlen;
+  }
   if ((int64_t)batch * hkv > 65535) return fail(ATTN_ERR_UNSUPPORTED, "batch * hkv must be <= 65535");
-  if ((int64_t)batch * hkv * d * fp8_vt_pitch(seqlen) > ((int64_t)1 << 40))
+  if ((int64_t)batch * hkv * d * fp8_vt_pitch(max_seqlen) > ((int64_t)1 << 40))
     return fail(ATTN_ERR_UNSUPPORTED, "problem too large for this library");
-  return check_shapes(nullptr, batch, seqlen, seqlen, batch * seqlen, hq, hkv, d, scale, causal, ATTN_BF16, pb);
+  return check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal, ATTN_BF16, pb);
 }
 }  // namespace
 
@@ -262,30 +269,48 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, const int32_t*
                    "attn_fwd (fp32 check mode) launch");
 }
 
+attn_status attn_fp8_quantize_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                     int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
+                                     int32_t d, void* q8, void* k8, void* vt8, float* descale_q, float* descale_k,
+                                     float* descale_v, void* stream) {
+  Problem pb;
+  if (cu_seqlens == nullptr) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  attn_status st = check_fp8(cu_seqlens, batch, 0, max_seqlen, total_tokens, hq, hkv, d, 1.f, 0, &pb);
+  if (st != ATTN_OK) return st;
+  if (batch == 0 || total_tokens == 0) return ok();
+  if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) || (st = check_ptr(q8, "q8")) ||
+      (st = check_ptr(k8, "k8")) || (st = check_ptr(vt8, "vt8")) || (st = check_ptr(descale_q, "descale_q")) ||
+      (st = check_ptr(descale_k, "descale_k")) || (st = check_ptr(descale_v, "descale_v")))
+    return st;
+  return from_cuda(launch_fp8_quantize(q, k, v, cu_seqlens, batch, 0, max_seqlen, total_tokens, hq, hkv, d, q8, k8,
+                                       vt8, descale_q, descale_k, descale_v, static_cast<cudaStream_t>(stream)),
+                   "attn_fp8_quantize_varlen launch");
+}
+
 attn_status attn_fp8_quantize(const void* q, const void* k, const void* v, int32_t batch, int32_t seqlen, int32_t hq,
                               int32_t hkv, int32_t d, void* q8, void* k8, void* vt8, float* descale_q,
                               float* descale_k, float* descale_v, void* stream) {
   Problem pb;
-  attn_status st = check_fp8(batch, seqlen, hq, hkv, d, 1.f, 0, &pb);
+  attn_status st = check_fp8(nullptr, batch, seqlen, 0, 0, hq, hkv, d, 1.f, 0, &pb);
   if (st != ATTN_OK) return st;
   if (batch == 0 || seqlen == 0) return ok();
   if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) || (st = check_ptr(q8, "q8")) ||
       (st = check_ptr(k8, "k8")) || (st = check_ptr(vt8, "vt8")) || (st = check_ptr(descale_q, "descale_q")) ||
       (st = check_ptr(descale_k, "descale_k")) || (st = check_ptr(descale_v, "descale_v")))
     return st;
-  return from_cuda(launch_fp8_quantize(q, k, v, batch, seqlen, hq, hkv, d, q8, k8, vt8, descale_q, descale_k,
-                                       descale_v, static_cast<cudaStream_t>(stream)),
+  return from_cuda(launch_fp8_quantize(q, k, v, nullptr, batch, seqlen, seqlen, batch * seqlen, hq, hkv, d, q8, k8,
+                                       vt8, descale_q, descale_k, descale_v, static_cast<cudaStream_t>(stream)),
                    "attn_fp8_quantize launch");
 }
 
-attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* descale_q,
-                         const float* descale_k, const float* descale_v, int32_t batch, int32_t seqlen, int32_t hq,
-                         int32_t hkv, int32_t d, float scale, int32_t causal, void* o, float* lse, void* workspace,
-                         size_t workspace_bytes, void* stream) {
-  Problem pb;
-  attn_status st = check_fp8(batch, seqlen, hq, hkv, d, scale, causal, &pb);
-  if (st != ATTN_OK) return st;
-  if (batch == 0 || seqlen == 0) return ok();
+}  // extern "C"
+
+namespace {
+// The FP8 forward once the shapes are checked (pb) and the batch is not empty.
+attn_status fwd_fp8_checked(const Problem& pb, const void* q8, const void* k8, const void* vt8,
+                            const float* descale_q, const float* descale_k, const float* descale_v, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes, void* stream, const char* what) {
+  attn_status st;
   if ((st = check_ptr(q8, "q8")) || (st = check_ptr(k8, "k8")) || (st = check_ptr(vt8, "vt8")) ||
       (st = check_ptr(descale_q, "descale_q")) || (st = check_ptr(descale_k, "descale_k")) ||
       (st = check_ptr(descale_v, "descale_v")) || (st = check_ptr(o, "o")) || (st = check_ptr(lse, "lse")))
@@ -296,7 +321,36 @@ attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const 
   if ((st = check_ptr(workspace, "workspace"))) return st;
   return from_cuda(launch_fwd_fp8(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace,
                                   static_cast<cudaStream_t>(stream)),
-                   "attn_fwd_fp8 launch");
+                   what);
+}
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* descale_q,
+                         const float* descale_k, const float* descale_v, int32_t batch, int32_t seqlen, int32_t hq,
+                         int32_t hkv, int32_t d, float scale, int32_t causal, void* o, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Problem pb;
+  attn_status st = check_fp8(nullptr, batch, seqlen, 0, 0, hq, hkv, d, scale, causal, &pb);
+  if (st != ATTN_OK) return st;
+  if (batch == 0 || seqlen == 0) return ok();
+  return fwd_fp8_checked(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace, workspace_bytes, stream,
+                         "attn_fwd_fp8 launch");
+}
+
+attn_status attn_fwd_fp8_varlen(const void* q8, const void* k8, const void* vt8, const float* descale_q,
+                                const float* descale_k, const float* descale_v, const int32_t* cu_seqlens,
+                                int32_t batch, int32_t max_seqlen, int32_t total_tokens, int32_t hq, int32_t hkv,
+                                int32_t d, float scale, int32_t causal, void* o, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  Problem pb;
+  if (cu_seqlens == nullptr) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  attn_status st = check_fp8(cu_seqlens, batch, 0, max_seqlen, total_tokens, hq, hkv, d, scale, causal, &pb);
+  if (st != ATTN_OK) return st;
+  if (batch == 0 || total_tokens == 0) return ok();
+  return fwd_fp8_checked(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace, workspace_bytes, stream,
+                         "attn_fwd_fp8_varlen launch");
 }
 
 }  // extern "C"

@@ -5,8 +5,9 @@
 // here is per head: descale_x[h] = amax_h / 448 (448 = the largest e4m3 value), and
 // x8 = e4m3(x / descale_x[h]) (fp32 division, then rounded to nearest even with
 // saturation).  Q and K keep their [T, heads, d] layout; V is written transposed per
-// (sequence, head), vt8 [batch * hkv][d][pitch] (tokens contiguous, pitch = seqlen rounded
-// up to 16, zero-padded), the K-major B operand of the P V product.
+// (sequence, head), vt8 [batch * hkv][d][pitch] (tokens contiguous, pitch = the longest
+// sequence rounded up to 16, zero-padded), the K-major B operand of the P V product.
+// Sequences are fixed-length (batch x seqlen) or packed and described by cu_seqlens.
 #include <algorithm>
 
 #include "kernels.h"
@@ -78,10 +79,12 @@ __global__ void __launch_bounds__(256) quantize_rows(const __nv_bfloat16* __rest
   }
 }
 
-// vt8[b * hkv + g][c][t] = e4m3(v[b * seqlen + t][g][c] / descale[g]) for t < seqlen and 0
-// for seqlen <= t < pitch, through a 64-token x 64-feature shared tile so that both the
-// reads (along c) and the writes (along t) are coalesced.
-__global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16* __restrict__ v, int seqlen,
+// vt8[b * hkv + g][c][t] = e4m3(v[start_b + t][g][c] / descale[g]) for t < len_b and 0 for
+// len_b <= t < pitch (start_b, len_b from cu_seqlens, or b * seqlen and seqlen), through a
+// 64-token x 64-feature shared tile so that both the reads (along c) and the writes (along
+// t) are coalesced.
+__global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16* __restrict__ v,
+                                                             const int32_t* __restrict__ cu_seqlens, int seqlen,
                                                              int pitch, int hkv, int d, const float* __restrict__ descale,
                                                              uint8_t* __restrict__ vt8) {
   __shared__ __align__(4) uint8_t tile[64][64 + 4];
@@ -90,11 +93,15 @@ __global__ void __launch_bounds__(256) quantize_v_transposed(const __nv_bfloat16
   const int c0 = blockIdx.y * 64;
   const int t0 = blockIdx.x * 64;
   const float ds = descale[g];
+  const int start = cu_seqlens ? cu_seqlens[b] : b * seqlen;
+  // a length beyond the pitch (max_seqlen too small) is cut at the pitch; the forward
+  // reports that case
+  const int len = min(cu_seqlens ? cu_seqlens[b + 1] - start : seqlen, pitch);
   for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
     const int tt = e / 64, cc = e % 64;
     const int t = t0 + tt;
     float x = 0.f;
-    if (t < seqlen) x = __bfloat162float(v[(((size_t)b * seqlen + t) * hkv + g) * d + c0 + cc]);
+    if (t < len) x = __bfloat162float(v[(((size_t)start + t) * hkv + g) * d + c0 + cc]);
     tile[cc][tt] = to_e4m3(__fdiv_rn(x, ds));
   }
   __syncthreads();
@@ -120,12 +127,13 @@ int q8_sm_count() {
 
 }  // namespace
 
-cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int batch, int seqlen, int hq, int hkv,
-                                int d, void* q8, void* k8, void* vt8, float* descale_q, float* descale_k,
-                                float* descale_v, cudaStream_t stream) {
-  const int total_tokens = batch * seqlen;
-  if (total_tokens == 0 || d % 64 != 0) return total_tokens == 0 ? cudaSuccess : cudaErrorInvalidValue;
-  const int pitch = fp8_vt_pitch(seqlen);
+cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                                int seqlen, int max_seqlen, int total_tokens, int hq, int hkv, int d, void* q8,
+                                void* k8, void* vt8, float* descale_q, float* descale_k, float* descale_v,
+                                cudaStream_t stream) {
+  if (total_tokens == 0 || batch == 0 || d % 64 != 0)
+    return (total_tokens == 0 || batch == 0) ? cudaSuccess : cudaErrorInvalidValue;
+  const int pitch = fp8_vt_pitch(cu_seqlens ? max_seqlen : seqlen);
   const int grid = q8_sm_count() * 8;
   const int64_t nq = (int64_t)total_tokens * hq * d, nk = (int64_t)total_tokens * hkv * d;
   cudaError_t e;
@@ -153,8 +161,9 @@ cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int
   launch(amax_to_descale, dim3((hkv + 255) / 256), bv, hkv);
   launch(quantize_rows, dim3(grid), qb, nq, hq, d, static_cast<const float*>(descale_q), static_cast<uint8_t*>(q8));
   launch(quantize_rows, dim3(grid), kb, nk, hkv, d, static_cast<const float*>(descale_k), static_cast<uint8_t*>(k8));
-  launch(quantize_v_transposed, dim3((pitch + 63) / 64, d / 64, batch * hkv), vb, seqlen, pitch, hkv, d,
-         static_cast<const float*>(descale_v), static_cast<uint8_t*>(vt8));
+  if (pitch > 0)
+    launch(quantize_v_transposed, dim3((pitch + 63) / 64, d / 64, batch * hkv), vb, cu_seqlens, seqlen, pitch, hkv,
+           d, static_cast<const float*>(descale_v), static_cast<uint8_t*>(vt8));
   e = cudaGetLastError();
   return e;
 }

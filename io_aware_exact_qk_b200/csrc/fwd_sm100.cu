@@ -759,7 +759,7 @@ template <int D>
 cudaError_t launch_fwd_fp8_d(const Problem& pb, const void* q8, const void* k8, const void* vt8,
                              const float* descale_q, const float* descale_k, const float* descale_v, void* o,
                              float* lse, void* workspace, cudaStream_t stream) {
-  const int sp = fp8_vt_pitch(pb.seqlen);
+  const int sp = fp8_vt_pitch(pb.cu_seqlens ? pb.max_seqlen : pb.seqlen);
   alignas(64) CUtensorMap tq, tk, tv;
   // Q8, K8: [tokens, heads, d] bytes, one d-byte swizzled row per token
   if (!encode_tma_u8_3d(&tq, q8, D, pb.hq, pb.total_tokens, (uint64_t)D, (uint64_t)pb.hq * D, D, 1, kRows) ||
@@ -780,7 +780,6 @@ cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, co
                            const float* descale_q, const float* descale_k, const float* descale_v, void* o,
                            float* lse, void* workspace, cudaStream_t stream) {
   if (pb.total_tokens == 0 || pb.batch == 0 || pb.max_seqlen == 0) return cudaSuccess;
-  if (pb.cu_seqlens != nullptr) return cudaErrorInvalidValue;
   switch (pb.d) {
     case 64:
       return launch_fwd_fp8_d<64>(pb, q8, k8, vt8, descale_q, descale_k, descale_v, o, lse, workspace, stream);

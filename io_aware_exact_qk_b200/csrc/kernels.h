@@ -64,16 +64,19 @@ cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_par
                                  int total_tokens, int hq, int d, int first, cudaStream_t stream);
 cudaError_t launch_merge_finish(const float* o_acc, void* o, int total_tokens, int hq, int d, cudaStream_t stream);
 
-// FP8 forward (d = 64 or 128, fixed-length batches): e4m3 Q8, K8 [tokens, heads, d] and
-// V^T [batch * hkv][d][fp8_vt_pitch(seqlen)] with per-head descales; bf16 O, fp32 LSE.
+// FP8 forward (d = 64 or 128; fixed-length batches or cu_seqlens): e4m3 Q8, K8 [tokens,
+// heads, d] and V^T [batch * hkv][d][fp8_vt_pitch(max_seqlen)] with per-head descales;
+// bf16 O, fp32 LSE.
 inline int fp8_vt_pitch(int seqlen) { return (seqlen + 15) / 16 * 16; }
 cudaError_t launch_fwd_fp8(const Problem& pb, const void* q8, const void* k8, const void* vt8,
                            const float* descale_q, const float* descale_k, const float* descale_v, void* o,
                            float* lse, void* workspace, cudaStream_t stream);
-// Per-head e4m3 quantisation of bf16 Q, K, V (fixed-length batch) into those operands.
-cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, int batch, int seqlen, int hq, int hkv,
-                                int d, void* q8, void* k8, void* vt8, float* descale_q, float* descale_k,
-                                float* descale_v, cudaStream_t stream);
+// Per-head e4m3 quantisation of bf16 Q, K, V into those operands (cu_seqlens nullptr:
+// batch sequences of seqlen tokens; else packed sequences of at most max_seqlen tokens).
+cudaError_t launch_fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                                int seqlen, int max_seqlen, int total_tokens, int hq, int hkv, int d, void* q8,
+                                void* k8, void* vt8, float* descale_q, float* descale_k, float* descale_v,
+                                cudaStream_t stream);
 
 // fp32 check mode (SIMT fp32 arithmetic).
 cudaError_t launch_fwd_fp32(const Problem& pb, const float* q, const float* k, const float* v, float* o,

@@ -159,6 +159,31 @@ def test_fp8_calls_reject_bad_arguments_on_host(lib):
                                  None) == attn.ATTN_OK
 
 
+def _fwd_fp8_varlen(lib, d=128, cu=0x2000, batch=2, max_seqlen=64, total=100, ptr=0x1000, o=0x1000, wsb=256):
+    vp = ctypes.c_void_p
+    return lib.attn_fwd_fp8_varlen(vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(ptr), vp(cu), batch, max_seqlen,
+                                   total, 2, 2, d, ctypes.c_float(0.1), 1, vp(o), vp(ptr), vp(0x1000), wsb, None)
+
+
+def test_fp8_varlen_calls_reject_bad_arguments_on_host(lib):
+    assert _fwd_fp8_varlen(lib, cu=None) == attn.ATTN_ERR_INVALID_ARG              # the packed calls need it
+    assert _fwd_fp8_varlen(lib, max_seqlen=101) == attn.ATTN_ERR_INVALID_ARG       # longer than all tokens
+    assert _fwd_fp8_varlen(lib, total=-1) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(lib, d=32) == attn.ATTN_ERR_UNSUPPORTED
+    assert _fwd_fp8_varlen(lib, o=0x1004) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(lib, wsb=8) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(lib, total=0, max_seqlen=0, ptr=None, o=None) == attn.ATTN_OK   # empty: no-op
+    vp = ctypes.c_void_p
+    p = vp(0x1000)
+    q8v = lib.attn_fp8_quantize_varlen
+    assert q8v(p, p, p, None, 2, 64, 100, 2, 2, 128, p, p, p, p, p, p, None) == attn.ATTN_ERR_INVALID_ARG
+    assert q8v(p, p, p, vp(0x2000), 2, 64, 100, 2, 2, 64 + 32, p, p, p, p, p, p, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert q8v(p, p, p, vp(0x2000), 2, 64, 100, 2, 2, 128, p, p, None, p, p, p, None) == attn.ATTN_ERR_INVALID_ARG
+    assert q8v(p, p, p, vp(0x2002), 2, 64, 100, 2, 2, 128, p, p, p, p, p, p, None) == attn.ATTN_ERR_INVALID_ARG
+    assert q8v(None, None, None, vp(0x2000), 2, 0, 0, 2, 2, 128, None, None, None, None, None, None,
+               None) == attn.ATTN_OK
+
+
 def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
     """include/attn.h is a C header (C99, no C++), and a C program links libattn.so and
     gets the host-side answers (workspace sizes, validation statuses) without a GPU."""

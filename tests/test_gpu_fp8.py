@@ -54,6 +54,18 @@ def transpose_v_cpu(v8, batch, seqlen):
     return out
 
 
+def transpose_v_cpu_varlen(v8, cu, max_seqlen):
+    """v8 [T, hkv, d] packed by cu_seqlens -> [batch hkv, d, pitch(max_seqlen)]: sequence b's
+    tokens at columns 0 .. len_b - 1, zeros after them."""
+    T, hkv, d = v8.shape
+    batch = len(cu) - 1
+    out = torch.zeros(batch, hkv, d, pitch_of(max_seqlen), dtype=torch.uint8)
+    for b in range(batch):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        out[b, :, :, :s1 - s0] = v8[s0:s1].permute(1, 2, 0)
+    return out.reshape(batch * hkv, d, pitch_of(max_seqlen))
+
+
 def dequant(x8, ds):
     return x8.view(torch.float8_e4m3fn).double() * ds.double()[None, :, None]
 
@@ -200,3 +212,87 @@ def test_fp8_forward_bench_size_sampled_heads(causal):
         o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd[rows, h:h + 1], kd[rows, h:h + 1], vd[rows, h:h + 1],
                                                 scale=w.scale, causal=causal)
         parity.check_fwd_bf16(o[rows, h:h + 1], lse[h:h + 1, rows], o_ref, lse_ref, tag=f"fp8 b{b} h{h}")
+
+
+VARLEN_CASES = [
+    # name, sequence lengths, hq, hkv, causal, seed, d
+    ("fp8-varlen-gqa", [100, 700, 300, 1, 129], 4, 2, False, 51, 128),
+    ("fp8-varlen-gqa-causal", [100, 700, 300, 1, 129], 4, 2, True, 52, 128),
+    ("fp8-varlen-d64-causal", [513, 64, 1000, 17], 8, 2, True, 53, 64),
+    ("fp8-varlen-d64", [256, 255, 2], 2, 1, False, 54, 64),
+    ("fp8-varlen-empty-seq", [300, 0, 130], 2, 2, True, 55, 128),
+]
+
+
+def fp8_varlen_case(case):
+    name, lens, hq, hkv, causal, seed, d = case
+    w = W.custom(name, lens, hq, hkv, d, causal, seed)
+    q, k, v, _, cu = W.make_inputs(w, with_grad=False)
+    return w, q, k, v, cu
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=[c[0] for c in VARLEN_CASES])
+def test_fp8_quantize_varlen_bit_exact(case):
+    """Packed sequences: Q8 / K8 / descales as for a fixed-length batch; V^T per (sequence,
+    kv head) with the longest sequence's pitch and each shorter sequence zero-padded."""
+    w, q, k, v, cu = fp8_varlen_case(case)
+    dev = torch.device("cuda")
+    q8, k8, vt8, dq, dk, dv = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), cu_seqlens=cu.to(dev),
+                                                     max_seqlen=w.max_seqlen)
+    attn.attn_get_device_error()
+    q8_ref, dq_ref = quantize_cpu(q, w.hq)
+    k8_ref, dk_ref = quantize_cpu(k, w.hkv)
+    v8_ref, dv_ref = quantize_cpu(v, w.hkv)
+    assert torch.equal(dq.cpu(), dq_ref) and torch.equal(dk.cpu(), dk_ref) and torch.equal(dv.cpu(), dv_ref)
+    assert torch.equal(q8.cpu(), q8_ref) and torch.equal(k8.cpu(), k8_ref)
+    assert tuple(vt8.shape) == (w.batch * w.hkv, w.d, pitch_of(w.max_seqlen))
+    assert torch.equal(vt8.cpu(), transpose_v_cpu_varlen(v8_ref, cu.tolist(), w.max_seqlen))
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=[c[0] for c in VARLEN_CASES])
+def test_fp8_forward_varlen_matches_oracle(case):
+    """The FP8 forward over packed sequences, on operands quantised here on the CPU."""
+    w, q, k, v, cu = fp8_varlen_case(case)
+    q8, dq = quantize_cpu(q, w.hq)
+    k8, dk = quantize_cpu(k, w.hkv)
+    v8, dv = quantize_cpu(v, w.hkv)
+    vt8 = transpose_v_cpu_varlen(v8, cu.tolist(), w.max_seqlen)
+    dev = torch.device("cuda")
+    o, lse = attn.attn_fwd_fp8(q8.to(dev), k8.to(dev), vt8.to(dev), dq.to(dev), dk.to(dev), dv.to(dev),
+                               cu_seqlens=cu.to(dev), max_seqlen=w.max_seqlen, scale=w.scale, causal=w.causal)
+    attn.attn_get_device_error()
+    o, lse = parity.to_np(o), parity.to_np(lse)
+    qd, kd, vd = dequant(q8, dq).numpy(), dequant(k8, dk).numpy(), dequant(v8, dv).numpy()
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd, kd, vd, cu.numpy(), scale=w.scale, causal=w.causal)
+    parity.check_fwd_bf16(o, lse, o_ref, lse_ref, tag=w.name)
+    o_ex, _ = oracle.attn_fwd(qd, kd, vd, cu.numpy(), scale=w.scale, causal=w.causal)
+    assert parity.rel_l2(o, o_ex) <= FP8_EXACT_REL_L2, w.name
+
+
+def test_fp8_varlen_end_to_end_through_quantize():
+    """attn_fp8_quantize then attn_fwd_fp8 on packed sequences, both on the device."""
+    w, q, k, v, cu = fp8_varlen_case(("fp8-varlen-e2e", [384, 1000, 5, 640], 4, 2, True, 56, 128))
+    dev = torch.device("cuda")
+    cu_d = cu.to(dev)
+    ops = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), cu_seqlens=cu_d, max_seqlen=w.max_seqlen)
+    o, lse = attn.attn_fwd_fp8(*ops, cu_seqlens=cu_d, max_seqlen=w.max_seqlen, scale=w.scale, causal=True)
+    attn.attn_get_device_error()
+    q8, dq = quantize_cpu(q, w.hq)
+    k8, dk = quantize_cpu(k, w.hkv)
+    v8, dv = quantize_cpu(v, w.hkv)
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(dequant(q8, dq).numpy(), dequant(k8, dk).numpy(),
+                                            dequant(v8, dv).numpy(), cu.numpy(), scale=w.scale, causal=True)
+    parity.check_fwd_bf16(parity.to_np(o), parity.to_np(lse), o_ref, lse_ref, tag=w.name)
+
+
+def test_fp8_varlen_sequence_longer_than_max_seqlen_is_reported():
+    """As for the bf16 forward: a max_seqlen below the longest sequence is reported through
+    attn_get_device_error, not silently truncated."""
+    w, q, k, v, cu = fp8_varlen_case(("fp8-varlen-short", [100, 700, 300], 4, 2, True, 57, 128))
+    dev = torch.device("cuda")
+    cu_d = cu.to(dev)
+    ops = attn.attn_fp8_quantize(q.to(dev), k.to(dev), v.to(dev), cu_seqlens=cu_d, max_seqlen=512)
+    attn.attn_fwd_fp8(*ops, cu_seqlens=cu_d, max_seqlen=512, scale=w.scale, causal=True)
+    with pytest.raises(attn.AttnError) as e:
+        attn.attn_get_device_error()
+    assert e.value.status == attn.ATTN_ERR_INVALID_ARG
