@@ -50,10 +50,11 @@ class Workload:
     seed: int
     lengths: Optional[tuple] = None   # varlen: per-sequence lengths
     qk_mult: float = 1.0              # stability variant: Q and K multiplied before rounding
+    scale_arg: Optional[float] = None   # the score scale if not 1/sqrt(d)
 
     @property
     def scale(self) -> float:
-        return 1.0 / math.sqrt(self.d)
+        return self.scale_arg if self.scale_arg is not None else 1.0 / math.sqrt(self.d)
 
     @property
     def seqlens(self) -> List[int]:
@@ -125,10 +126,12 @@ def long32k() -> Workload:
     return Workload("long32k", 1, 32768, 16, 16, 128, True, seed=1006)
 
 
-def custom(name, seqlens, hq, hkv, d, causal, seed, qk_mult=1.0) -> Workload:
-    """Any other shape (tests use this for ragged and edge cases)."""
+def custom(name, seqlens, hq, hkv, d, causal, seed, qk_mult=1.0, scale=None) -> Workload:
+    """Any other shape (tests use this for ragged and edge cases, and for a score scale
+    other than 1/sqrt(d))."""
     seqlens = tuple(int(n) for n in seqlens)
-    return Workload(name, len(seqlens), 0, hq, hkv, d, causal, seed, lengths=seqlens, qk_mult=qk_mult)
+    return Workload(name, len(seqlens), 0, hq, hkv, d, causal, seed, lengths=seqlens, qk_mult=qk_mult,
+                    scale_arg=scale)
 
 
 def make_inputs(w: Workload, dtype: torch.dtype = torch.bfloat16, with_grad: bool = True):

@@ -102,3 +102,31 @@ def test_accumulate_mode_adds_float32_gradients(d, causal):
     bf = [P.to_np(t) for t in attn.attn_bwd(qd, kd, vd, o, dod, lse, **kw)]
     for name, a, b in zip(("dq", "dk", "dv"), once, bf):
         assert np.abs(a - b).max() <= 2 ** -8 * np.abs(a).max() + 1e-6, name
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.25])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_explicit_scale_and_three_heads_per_group(scale, d, causal):
+    """The score scale is a free argument (here 0.05 and 0.25 instead of 1/sqrt(d)), with
+    three query heads per K/V head and ragged sequences: forward and backward against the
+    oracle at the same scale."""
+    w = W.custom(f"scale{scale}_d{d}", [1, 129, 300, 64], 6, 2, d, causal, seed=95 + d, scale=scale)
+    q, k, v, do, cu = W.make_inputs(w)
+    o, lse = P.gpu_fwd(w, q, k, v, cu)
+    o_ref, lse_ref = P.oracle_fwd(w, q, k, v, cu)
+    P.check_fwd_bf16(P.to_np(o), P.to_np(lse), o_ref, lse_ref, tag=w.name)
+    grads = P.gpu_bwd(w, q, k, v, o.cpu(), do, lse.cpu(), cu)
+    ref = P.oracle_bwd(w, q, k, v, do, cu)
+    P.check_grads_bf16(grads, ref[:3], tag=w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp32_check_mode_explicit_scale(causal):
+    """The fp32 check mode at a scale other than 1/sqrt(d), three heads per group."""
+    w = W.custom("fp32_scale", [1, 77, 150], 6, 2, 64, causal, seed=99, scale=0.3)
+    grads, ref = _run(w, dtype=torch.float32)
+    for name, g, r in zip(("dq", "dk", "dv"), grads, ref[:3]):
+        g = P.to_np(g)
+        assert P.rel_l2(g, r) <= P.FP32_REL, name
+        assert P.max_rel(g, r) <= P.FP32_REL, name
