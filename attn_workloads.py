@@ -166,10 +166,11 @@ class DecodeWorkload:
     causal: bool
     seed: int
     random_k: Optional[tuple] = None   # (lo, hi): k_lens drawn from the seed stream first
+    scale_arg: Optional[float] = None   # the score scale if not 1/sqrt(d)
 
     @property
     def scale(self) -> float:
-        return 1.0 / math.sqrt(self.d)
+        return self.scale_arg if self.scale_arg is not None else 1.0 / math.sqrt(self.d)
 
     @property
     def batch(self) -> int:
@@ -220,8 +221,9 @@ def decode_spec4() -> DecodeWorkload:
     return DecodeWorkload("decode_spec4", (4,) * 16, (4096,) * 16, 32, 8, 128, True, seed=1103)
 
 
-def decode_custom(name, q_lens, k_lens, hq, hkv, d, causal, seed) -> DecodeWorkload:
-    return DecodeWorkload(name, tuple(int(x) for x in q_lens), tuple(int(x) for x in k_lens), hq, hkv, d, causal, seed)
+def decode_custom(name, q_lens, k_lens, hq, hkv, d, causal, seed, scale=None) -> DecodeWorkload:
+    return DecodeWorkload(name, tuple(int(x) for x in q_lens), tuple(int(x) for x in k_lens), hq, hkv, d, causal, seed,
+                          scale_arg=scale)
 
 
 def make_decode_inputs(w: DecodeWorkload, dtype: torch.dtype = torch.bfloat16):

@@ -49,8 +49,8 @@ def check(w, o, lse, o_ref, lse_ref, tag):
         assert e_lse <= parity.BF16_LSE_MAX_ABS, f"{tag} max|dLSE| {e_lse}"
 
 
-def case(name, q_lens, k_lens, hq, hkv, d, causal, seed, splits=(0,), varlen=True):
-    w = W.decode_custom(name, q_lens, k_lens, hq, hkv, d, causal, seed)
+def case(name, q_lens, k_lens, hq, hkv, d, causal, seed, splits=(0,), varlen=True, scale=None):
+    w = W.decode_custom(name, q_lens, k_lens, hq, hkv, d, causal, seed, scale=scale)
     q, k, v, cu_q, cu_k = W.make_decode_inputs(w)
     o_ref, lse_ref = oracle.attn_fwd_cross(q, k, v, cu_q.numpy(), cu_k.numpy(), scale=w.scale, causal=causal)
     for s in splits:
@@ -86,6 +86,12 @@ def test_more_query_rows_than_keys_leaves_early_rows_empty():
 def test_full_tile_of_rows_and_mha():
     case("rows128", [4, 4], [600, 333], 32, 1, 128, True, 2006, splits=(0, 3))      # 32 heads x 4 rows = 128
     case("mha_one_row", [1, 1], [777, 1500], 4, 4, 64, False, 2007, splits=(0, 4))  # one row per tile
+
+
+@pytest.mark.parametrize("scale", [0.04, 0.3])
+def test_explicit_scale_three_heads_per_group(scale):
+    # a score scale other than 1/sqrt(d), 3 query heads per KV head, causal speculative rows
+    case(f"scale{scale}", [2, 3, 1], [700, 65, 2000], 6, 2, 128, True, 2010, splits=(0, 1, 3), scale=scale)
 
 
 def test_varlen_query_lengths_differ():

@@ -150,6 +150,25 @@ def test_fp8_forward_matches_oracle(case):
     assert np.abs(lse - lse_ex).max() <= parity.BF16_LSE_MAX_ABS, name
 
 
+@pytest.mark.parametrize("scale", [0.03, 0.3])
+def test_fp8_forward_explicit_scale(scale):
+    """A score scale other than 1/sqrt(d) (it multiplies the two descales in the kernel),
+    three query heads per K/V head, packed sequences."""
+    w = W.custom(f"fp8-scale{scale}", [300, 129, 513], 6, 2, 128, True, 58, scale=scale)
+    q, k, v, _, cu = W.make_inputs(w, with_grad=False)
+    q8, dq = quantize_cpu(q, w.hq)
+    k8, dk = quantize_cpu(k, w.hkv)
+    v8, dv = quantize_cpu(v, w.hkv)
+    vt8 = transpose_v_cpu_varlen(v8, cu.tolist(), w.max_seqlen)
+    dev = torch.device("cuda")
+    o, lse = attn.attn_fwd_fp8(q8.to(dev), k8.to(dev), vt8.to(dev), dq.to(dev), dk.to(dev), dv.to(dev),
+                               cu_seqlens=cu.to(dev), max_seqlen=w.max_seqlen, scale=scale, causal=True)
+    attn.attn_get_device_error()
+    qd, kd, vd = dequant(q8, dq).numpy(), dequant(k8, dk).numpy(), dequant(v8, dv).numpy()
+    o_ref, lse_ref = oracle.attn_fwd_fp8sim(qd, kd, vd, cu.numpy(), scale=scale, causal=True)
+    parity.check_fwd_bf16(parity.to_np(o), parity.to_np(lse), o_ref, lse_ref, tag=w.name)
+
+
 def test_fp8_forward_large_scores_and_uneven_scales():
     """Q and K four times larger (scores of ~±20 in log2 units: the running max moves in
     large jumps and stays stale by up to 8) and per-head scales that differ by orders of
