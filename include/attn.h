@@ -145,6 +145,38 @@ attn_status attn_bwd_noalloc(const void *q, const void *k, const void *v,
                              float scale, int32_t causal, int32_t dtype,
                              void *dq, void *dk, void *dv, void *stream);
 
+/* One forward and one backward on HOST buffers, with the host <-> device copies overlapped
+ * with the kernels: attn_fwd then attn_bwd (the tutorial's 前向 and 反向重算流程) for callers
+ * whose tensors live in host memory.
+ *   q, k, v, dout (inputs) and o, lse, dq, dk, dv (outputs): HOST arrays in the layouts of
+ *       attn_fwd / attn_bwd (bf16; lse float32 [hq, total_tokens]); they should be
+ *       page-locked (cudaHostAlloc / cudaHostRegister), or the copies overlap nothing;
+ *   cu_seqlens: NULL (batch sequences of seqlen tokens) or a HOST int32 array [batch + 1]
+ *       starting at 0, ending at total_tokens, never decreasing, no step above max_seqlen;
+ *   scratch: caller-owned DEVICE memory of attn_fwd_bwd_host_scratch_size() bytes, 16-byte
+ *       aligned (the device copies of all tensors, the groups' cu_seqlens, and one forward
+ *       and one backward workspace).
+ * The sequences are split into up to four groups of whole sequences with about equal token
+ * counts; on three streams of the library's own, each group's rows are copied in, its
+ * forward and backward run, and its results are copied out while the other groups copy.
+ * Results are those of attn_fwd / attn_bwd on each group (O, LSE, dK, dV bit-identical to a
+ * single call on all sequences; dQ up to the order of its fp32 sums).  Ordering: the first
+ * copy waits for the work queued on `stream` before the call, and work queued on `stream`
+ * afterwards waits for the last copy; the host outputs are complete once `stream` is
+ * synchronised; calls that share a scratch must be ordered (one stream, or events), as calls
+ * on one stream are.  Enqueueing is serialised per device.  Errors: those of attn_fwd / attn_bwd
+ * and ATTN_ERR_INVALID_ARG for a malformed cu_seqlens, a NULL host array or a small or
+ * unaligned scratch, all found on the host before anything is queued; a failing CUDA call
+ * returns ATTN_ERR_CUDA after the part of the pipeline already queued has finished. */
+size_t attn_fwd_bwd_host_scratch_size(int32_t batch, int32_t total_tokens,
+                                      int32_t hq, int32_t hkv, int32_t d);
+attn_status attn_fwd_bwd_host(const void *q, const void *k, const void *v, const void *dout,
+                              const int32_t *cu_seqlens, int32_t batch, int32_t seqlen,
+                              int32_t max_seqlen, int32_t total_tokens,
+                              int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal,
+                              void *o, float *lse, void *dq, void *dk, void *dv,
+                              void *scratch, size_t scratch_bytes, void *stream);
+
 /* Decoding forward (split-KV).  The tutorial's FlashDecoding variant (section
  * "FlashAttention 变体族谱": one query against a long KV, the KV cut into blocks whose
  * partial results are computed in parallel and then reduced; section "变体选择场景":

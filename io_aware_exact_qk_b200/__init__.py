@@ -86,6 +86,10 @@ def load_library():
     lib.attn_fp8_quantize.restype = ctypes.c_int
     lib.attn_fwd_fp8.argtypes = [vp] * 6 + [i32] * 5 + [f32, i32, vp, vp, vp, sz, vp]
     lib.attn_fwd_fp8.restype = ctypes.c_int
+    lib.attn_fwd_bwd_host_scratch_size.argtypes = [i32] * 5
+    lib.attn_fwd_bwd_host_scratch_size.restype = sz
+    lib.attn_fwd_bwd_host.argtypes = [vp] * 5 + [i32] * 7 + [f32, i32] + [vp] * 6 + [sz, vp]
+    lib.attn_fwd_bwd_host.restype = ctypes.c_int
     lib.attn_fp8_quantize_varlen.argtypes = [vp, vp, vp, vp] + [i32] * 6 + [vp] * 6 + [vp]
     lib.attn_fp8_quantize_varlen.restype = ctypes.c_int
     lib.attn_fwd_fp8_varlen.argtypes = [vp] * 7 + [i32] * 6 + [f32, i32, vp, vp, vp, sz, vp]
@@ -402,37 +406,41 @@ def attn_launch_count():
     return int(load_library().attn_launch_count())
 
 
+def attn_fwd_bwd_host(q, k, v, do, cu_seqlens=None, max_seqlen=None, scale=None, causal=False, batch=None,
+                      out=None, scratch=None, stream=None):
+    """Forward and backward on HOST tensors (bf16 q [T,Hq,d], k, v [T,Hkv,d], do [T,Hq,d],
+    ideally pinned; cu_seqlens a host int32 tensor or None) through the library's own
+    copy/compute pipeline.  Returns ((o, lse, dq, dk, dv) host tensors, scratch); ``out``
+    may hold those five host tensors (pinned) and ``scratch`` the device scratch from a
+    previous call."""
+    lib = load_library()
+    b, seqlen, ms, T, hq, hkv, d = _shape_args(q, k, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
+               torch.empty(hq, T, dtype=torch.float32, pin_memory=True),
+               torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
+               torch.empty(k.shape, dtype=k.dtype, pin_memory=True),
+               torch.empty(v.shape, dtype=v.dtype, pin_memory=True))
+    need = int(lib.attn_fwd_bwd_host_scratch_size(b, T, hq, hkv, d))
+    if scratch is None:
+        scratch = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    cu = None if cu_seqlens is None else cu_seqlens.to(torch.int32).contiguous()
+    o, lse, dq, dk, dv = out
+    _check(lib.attn_fwd_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu), b, seqlen, ms, T, hq, hkv, d,
+                                 float(scale), int(bool(causal)), _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(scratch), scratch.numel(), _stream(stream)))
+    return out, scratch
+
+
 def attention_host(q, k, v, do, cu_seqlens=None, max_seqlen=None, scale=None, causal=False, batch=None,
-                   device=None, stream=None, out=None):
-    """Forward and backward on HOST tensors: copies q, k, v, do (ideally pinned) to the
-    device, runs attn_fwd and attn_bwd there, and copies O, LSE, dQ, dK, dV back into host
-    tensors.  Returns (o, lse, dq, dk, dv) on the host.  ``out`` may hold preallocated
-    device and pinned host buffers (a dict from a previous call) to avoid reallocation."""
-    device = torch.device("cuda") if device is None else device
+                   stream=None, out=None):
+    """attn_fwd_bwd_host with its buffers kept in a dict: returns ((o, lse, dq, dk, dv) on
+    the host, bufs); passing ``out=bufs`` from a previous call reuses the pinned outputs and
+    the device scratch."""
     bufs = out if out is not None else {}
-    if not bufs:
-        for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
-            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=device)
-        bufs["cu"] = None if cu_seqlens is None else torch.empty(cu_seqlens.shape, dtype=torch.int32, device=device)
-        T, hq, _ = q.shape
-        bufs["o"] = torch.empty_like(bufs["q"])
-        bufs["lse"] = torch.empty(hq, T, dtype=torch.float32, device=device)
-        bufs["dq"] = torch.empty_like(bufs["q"])
-        bufs["dk"] = torch.empty_like(bufs["k"])
-        bufs["dv"] = torch.empty_like(bufs["v"])
-        ws = max(workspace_size("fwd", q, k, cu_seqlens, max_seqlen, batch),
-                 workspace_size("bwd", q, k, cu_seqlens, max_seqlen, batch))
-        bufs["ws"] = torch.empty(max(ws, 1), dtype=torch.uint8, device=device)
-        for name in ("o", "lse", "dq", "dk", "dv"):
-            bufs["host_" + name] = torch.empty(bufs[name].shape, dtype=bufs[name].dtype, pin_memory=True)
-    for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
-        bufs[name].copy_(t, non_blocking=True)
-    if cu_seqlens is not None:
-        bufs["cu"].copy_(cu_seqlens, non_blocking=True)
-    attn_fwd(bufs["q"], bufs["k"], bufs["v"], bufs["cu"], max_seqlen, scale, causal, batch,
-             o=bufs["o"], lse=bufs["lse"], stream=stream)
-    attn_bwd(bufs["q"], bufs["k"], bufs["v"], bufs["o"], bufs["do"], bufs["lse"], bufs["cu"], max_seqlen, scale,
-             causal, batch, dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], workspace=bufs["ws"], stream=stream)
-    for name in ("o", "lse", "dq", "dk", "dv"):
-        bufs["host_" + name].copy_(bufs[name], non_blocking=True)
-    return tuple(bufs["host_" + n] for n in ("o", "lse", "dq", "dk", "dv")), bufs
+    res, bufs["scratch"] = attn_fwd_bwd_host(q, k, v, do, cu_seqlens, max_seqlen, scale, causal, batch,
+                                             out=bufs.get("host"), scratch=bufs.get("scratch"), stream=stream)
+    bufs["host"] = res
+    return res, bufs

@@ -116,6 +116,14 @@ std::atomic<int64_t> g_launches{0};
 
 }  // namespace
 
+int validate_shapes(const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen, int32_t total_tokens,
+                    int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal, int32_t dtype, Problem* pb) {
+  return check_shapes(cu_seqlens, batch, seqlen, max_seqlen, total_tokens, hq, hkv, d, scale, causal, dtype, pb);
+}
+int validate_ptr(const void* p, const char* name) { return check_ptr(p, name); }
+int cuda_status(cudaError_t e, const char* what) { return from_cuda(e, what); }
+int status_ok() { return ok(); }
+
 int record_error(int status, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);

@@ -129,6 +129,15 @@ int bwd_check_args(const void* q, const void* k, const void* v, const void* o, c
 // Records `fmt` as the calling thread's last error message (attn_last_error_message) and
 // returns `status`.
 int record_error(int status, const char* fmt, ...);
+// The entry points' shared host checks, for entry points in other files (each returns an
+// attn_status value and, on failure, records the reason): shape arguments (fills `pb`), a
+// device pointer (non-NULL, 16-byte aligned), a CUDA result, and success (clears the
+// message).
+int validate_shapes(const int32_t* cu_seqlens, int32_t batch, int32_t seqlen, int32_t max_seqlen, int32_t total_tokens,
+                    int32_t hq, int32_t hkv, int32_t d, float scale, int32_t causal, int32_t dtype, Problem* pb);
+int validate_ptr(const void* p, const char* name);
+int cuda_status(cudaError_t e, const char* what);
+int status_ok();
 
 // Host helper shared by the launchers: encodes a 3-D bf16 TMA descriptor over a
 // [rows, heads, d] tensor with a (box_inner x 1 x box_rows) box and the swizzle that

@@ -184,6 +184,32 @@ def test_fp8_varlen_calls_reject_bad_arguments_on_host(lib):
                None) == attn.ATTN_OK
 
 
+def test_host_step_rejects_bad_arguments_on_host(lib):
+    """attn_fwd_bwd_host checks its shapes, its host cu_seqlens and its scratch before it
+    touches the GPU."""
+    vp = ctypes.c_void_p
+    p = vp(0x1000)
+
+    def call(cu=None, batch=3, seqlen=100, max_seqlen=0, total=300, hq=4, hkv=2, d=128, ptr=p, scratch=p,
+             scratch_bytes=1 << 40):
+        return lib.attn_fwd_bwd_host(ptr, ptr, ptr, ptr, cu, batch, seqlen, max_seqlen, total, hq, hkv, d,
+                                     ctypes.c_float(0.1), 1, ptr, ptr, ptr, ptr, ptr, scratch, scratch_bytes, None)
+
+    assert call(hq=3) == attn.ATTN_ERR_UNSUPPORTED
+    assert call(total=299) == attn.ATTN_ERR_INVALID_ARG                       # batch * seqlen mismatch
+    assert call(ptr=None) == attn.ATTN_ERR_INVALID_ARG                        # NULL host arrays
+    assert call(scratch_bytes=1000) == attn.ATTN_ERR_INVALID_ARG              # scratch too small
+    assert b"scratch" in lib.attn_last_error_message()
+    assert call(scratch=vp(0x1008)) == attn.ATTN_ERR_INVALID_ARG              # unaligned scratch
+    cu_bad = [(0, 100, 50, 300), (0, 100, 200, 299), (1, 100, 200, 300), (0, 250, 260, 300)]
+    for vals in cu_bad:                                # decreasing, wrong end, wrong start, > max
+        arr = (ctypes.c_int32 * 4)(*vals)
+        assert call(cu=ctypes.cast(arr, vp), seqlen=0, max_seqlen=200) == attn.ATTN_ERR_INVALID_ARG, vals
+    assert call(batch=0, total=0, ptr=None, scratch=None, scratch_bytes=0) == attn.ATTN_OK   # empty: no-op
+    need = lib.attn_fwd_bwd_host_scratch_size(3, 300, 4, 2, 128)
+    assert need >= 300 * (4 * 4 + 4 * 2) * 128 * 2 + 300 * 4 * 4 * 128   # the tensors plus dQ's accumulator
+
+
 def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
     """include/attn.h is a C header (C99, no C++), and a C program links libattn.so and
     gets the host-side answers (workspace sizes, validation statuses) without a GPU."""
