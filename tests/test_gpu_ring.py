@@ -21,7 +21,8 @@ import torch.distributed as dist
 import attn_workloads as W
 import io_aware_exact_qk_b200 as attn
 import oracle
-from io_aware_exact_qk_b200.ring import ring_attn_bwd, ring_attn_fwd, ring_schedule
+from io_aware_exact_qk_b200.ring import (ring_attn_bwd, ring_attn_fwd, ring_schedule, zigzag_schedule, zigzag_shard,
+                                         zigzag_unshard)
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -102,6 +103,54 @@ def test_emulated_ring_backward_matches_the_gradient(world, causal, d):
                             tag=f"ring bwd W={world}")
 
 
+@pytest.mark.parametrize("world,d", [(2, 128), (3, 64), (4, 128)])
+def test_emulated_zigzag_ring_causal(world, d):
+    """The zig-zag layout under the causal mask, ranks emulated in turn with the library's
+    kernels: each rank's hops of ``zigzag_schedule`` (attn_fwd on each (query half, K/V
+    half) pair, merged per query half), then its backward pairs adding into float32 sums
+    (dK / dV into the visiting block's halves); all rows against the oracle."""
+    batch, c, hq, hkv = 2, 128, 8, 2
+    N = 2 * world * c
+    w = W.custom("zz", [N] * batch, hq, hkv, d, True, 3400 + world)
+    q, k, v, do, cu = W.make_inputs(w)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, cu.numpy(), scale=w.scale, causal=True)
+    shard = [[zigzag_shard(t, batch, r, world).cuda() for r in range(world)] for t in (q, k, v, do)]
+    qs, ks, vs, dos = shard
+    os_, lses = [], []
+    for r in range(world):
+        o_acc = torch.empty(2, batch * c, hq, d, device="cuda")
+        lse_acc = torch.empty(2, hq, batch * c, device="cuda")
+        first = [True, True]
+        for s, pairs in enumerate(zigzag_schedule(r, world, True)):
+            j = (r - s) % world
+            for a, b, kind in pairs:
+                o_p, lse_p = attn.attn_fwd(qs[r][a], ks[j][b], vs[j][b], scale=w.scale, causal=kind == "causal",
+                                           batch=batch)
+                attn.attn_merge_partial(o_acc[a], lse_acc[a], o_p, lse_p, first=first[a])
+                first[a] = False
+        os_.append(attn.attn_merge_finish(o_acc.reshape(-1, hq, d)).reshape(2, batch * c, hq, d))
+        lses.append(lse_acc)
+    attn.attn_get_device_error()
+    o = zigzag_unshard([t.cpu() for t in os_], batch)
+    lse = zigzag_unshard([t.cpu().transpose(1, 2) for t in lses], batch).T
+    parity.check_fwd_bf16(parity.to_np(o), parity.to_np(lse), o_ref, lse_ref, tag=f"zigzag W={world}")
+    # backward on the device forward's O and LSE, as a caller of ring_attn_bwd would
+    dq = [torch.zeros(2, batch * c, hq, d, device="cuda") for _ in range(world)]
+    dk = [torch.zeros(2, batch * c, hkv, d, device="cuda") for _ in range(world)]
+    dv = [torch.zeros(2, batch * c, hkv, d, device="cuda") for _ in range(world)]
+    for r in range(world):
+        for s, pairs in enumerate(zigzag_schedule(r, world, True)):
+            j = (r - s) % world
+            for a, b, kind in pairs:
+                attn.attn_bwd_accumulate(qs[r][a], ks[j][b], vs[j][b], os_[r][a], dos[r][a],
+                                         lses[r][a].contiguous(), dq[r][a], dk[j][b], dv[j][b], scale=w.scale,
+                                         causal=kind == "causal", batch=batch)
+    attn.attn_get_device_error()
+    ref = oracle.attn_bwd(q, k, v, do, cu.numpy(), scale=w.scale, causal=True)
+    got = tuple(zigzag_unshard([t.cpu() for t in g], batch) for g in (dq, dk, dv))
+    parity.check_grads_bf16(got, ref[:3], tag=f"zigzag bwd W={world}")
+
+
 def test_merge_kernel_edge_cases():
     T, hq, d = 37, 4, 128
     g = torch.Generator().manual_seed(5)
@@ -150,5 +199,17 @@ def test_driver_as_a_one_rank_nccl_group():
         dq_r, dk_r, dv_r, _, _ = oracle.attn_bwd(q, k, v, do, cu.numpy(), scale=w.scale, causal=True,
                                                  o=o_st.double().numpy(), lse=lse_st.double().numpy())
         parity.check_grads_bf16((dq, dk, dv), (dq_r, dk_r, dv_r), tag="one-rank ring bwd")
+        # the zig-zag layout through the same drivers (one rank: chunks 0 and 1)
+        qz, kz, vz, oz, doz = (zigzag_shard(t, batch, 0, 1).cuda() for t in (q, k, v, o_st, do))
+        o2, lse2 = ring_attn_fwd(qz, kz, vz, batch, scale=w.scale, causal=True, layout="zigzag")
+        attn.attn_get_device_error()
+        o2 = zigzag_unshard([o2.cpu()], batch)
+        lse2 = zigzag_unshard([lse2.cpu().transpose(1, 2)], batch).T
+        parity.check_fwd_bf16(o2, lse2, o_ref, lse_ref, tag="one-rank zigzag ring")
+        lsez = zigzag_shard(lse_st.T.contiguous(), batch, 0, 1).transpose(1, 2).contiguous().cuda()
+        dq2, dk2, dv2 = ring_attn_bwd(qz, kz, vz, oz, doz, lsez, batch, scale=w.scale, causal=True, layout="zigzag")
+        attn.attn_get_device_error()
+        got = tuple(zigzag_unshard([t.cpu()], batch) for t in (dq2, dk2, dv2))
+        parity.check_grads_bf16(got, (dq_r, dk_r, dv_r), tag="one-rank zigzag ring bwd")
     finally:
         dist.destroy_process_group()

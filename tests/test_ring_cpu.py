@@ -16,7 +16,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from io_aware_exact_qk_b200.ring import ring_schedule
+from io_aware_exact_qk_b200.ring import ring_schedule, zigzag_schedule, zigzag_shard, zigzag_unshard
 
 
 def _free_port():
@@ -50,8 +50,8 @@ def _merge64(o_acc, lse_acc, o_p, lse_p, first):
     lse_acc.copy_(m + torch.log(s))
 
 
-def _local_oracle_bwd(batch, scale, o, do, lse):
-    def f(q, k, v, causal, dq_acc, dk_acc, dv_acc):
+def _local_oracle_bwd(batch, scale):
+    def f(q, k, v, o, do, lse, causal, dq_acc, dk_acc, dv_acc):
         n = q.shape[0] // batch
         cu = np.arange(batch + 1, dtype=np.int32) * n
         dq, dk, dv, _, _ = oracle.attn_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), cu, scale=scale,
@@ -70,19 +70,22 @@ def _full_inputs(batch, N, hq, hkv, d):
     return q, k, v, do
 
 
-def _worker(rank, world, port, batch, n, hq, hkv, d, causal, out):
+def _worker(rank, world, port, batch, n, hq, hkv, d, causal, out, layout="contiguous"):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
         from io_aware_exact_qk_b200.ring import ring_attn_bwd, ring_attn_fwd
         q, k, v, do = _full_inputs(batch, world * n, hq, hkv, d)
-        mine = slice(rank * n, (rank + 1) * n)
-        qc, kc, vc, doc = (t[:, mine].reshape(batch * n, t.shape[2], d).contiguous() for t in (q, k, v, do))
+        if layout == "zigzag":
+            qc, kc, vc, doc = (zigzag_shard(t.reshape(-1, t.shape[2], d), batch, rank, world) for t in (q, k, v, do))
+        else:
+            mine = slice(rank * n, (rank + 1) * n)
+            qc, kc, vc, doc = (t[:, mine].reshape(batch * n, t.shape[2], d).contiguous() for t in (q, k, v, do))
         scale = 1.0 / np.sqrt(d)
         o, lse = ring_attn_fwd(qc, kc, vc, batch, scale=scale, causal=causal, local_fwd=_local_oracle(batch, scale),
-                               merge=_merge64, finish=lambda oa: oa, acc_dtype=torch.float64)
+                               merge=_merge64, finish=lambda oa: oa, acc_dtype=torch.float64, layout=layout)
         dq, dk, dv = ring_attn_bwd(qc, kc, vc, o, doc, lse, batch, scale=scale, causal=causal,
-                                   local_bwd=_local_oracle_bwd(batch, scale, o, doc, lse), finish=lambda a: a,
-                                   acc_dtype=torch.float64)
+                                   local_bwd=_local_oracle_bwd(batch, scale), finish=lambda a: a,
+                                   acc_dtype=torch.float64, layout=layout)
         out[rank] = (o.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy())
         dist.barrier()
     finally:
@@ -133,3 +136,75 @@ def test_ring_schedule_visits_every_block_once():
                 assert hops[0] == (r, "causal" if causal else "full")   # own block first
                 for j, kind in hops:
                     assert kind == ("full" if not causal or j < r else ("causal" if j == r else None))
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_ring_equals_full_attention(world, causal):
+    """The zig-zag layout (rank r holds chunks r and 2W-1-r of every sequence): the rows
+    of all ranks, put back in sequence order, equal the oracle's forward and gradient."""
+    batch, c, hq, hkv, d = 2, 3, 4, 2, 8
+    N = 2 * world * c
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as man:
+        out = man.dict()
+        procs = [ctx.Process(target=_worker, args=(r, world, port, batch, N // world, hq, hkv, d, causal, out,
+                                                   "zigzag"))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    q, k, v, do = _full_inputs(batch, N, hq, hkv, d)
+    cu = np.arange(batch + 1, dtype=np.int32) * N
+    dq_ref, dk_ref, dv_ref, o_ref, lse_ref = oracle.attn_bwd(
+        q.reshape(-1, hq, d).numpy(), k.reshape(-1, hkv, d).numpy(), v.reshape(-1, hkv, d).numpy(),
+        do.reshape(-1, hq, d).numpy(), cu, causal=causal)
+
+    def whole(i):
+        return zigzag_unshard([torch.from_numpy(res[r][i]) for r in range(world)], batch).numpy()
+
+    lse = zigzag_unshard([torch.from_numpy(res[r][1]).transpose(1, 2) for r in range(world)], batch).T.numpy()
+    np.testing.assert_allclose(whole(0), o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(whole(2), dq_ref, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(whole(3), dk_ref, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(whole(4), dv_ref, rtol=0, atol=1e-10)
+
+
+def test_zigzag_schedule_balances_the_causal_ring():
+    """Every (query chunk, K/V chunk) pair a rank can see is visited exactly once, with the
+    right mask, and under the causal mask every rank has 2W - 1 full and 2 diagonal blocks."""
+    for world in (1, 2, 3, 5):
+        for causal in (False, True):
+            for r in range(world):
+                hops = zigzag_schedule(r, world, causal)
+                assert len(hops) == world
+                seen = []
+                for s, pairs in enumerate(hops):
+                    j = (r - s) % world
+                    for a, b, kind in pairs:
+                        qc = (r, 2 * world - 1 - r)[a]
+                        kc = (j, 2 * world - 1 - j)[b]
+                        assert kind == ("full" if not causal or kc < qc else "causal"), (world, r, s, a, b)
+                        seen.append((qc, kc))
+                want = [(qc, kc) for qc in (r, 2 * world - 1 - r) for kc in range(2 * world)
+                        if not causal or kc <= qc]
+                assert sorted(seen) == sorted(want)
+                if causal:
+                    kinds = [k for pairs in hops for _, _, k in pairs]
+                    assert kinds.count("full") == 2 * world - 1 and kinds.count("causal") == 2
+
+
+def test_zigzag_shard_round_trip():
+    x = torch.arange(2 * 12 * 3 * 4, dtype=torch.float64).reshape(2 * 12, 3, 4)
+    for world in (1, 2, 3, 6):
+        parts = [zigzag_shard(x, 2, r, world) for r in range(world)]
+        assert all(p.shape == (2, 2 * 12 // (2 * world), 3, 4) for p in parts)
+        assert torch.equal(zigzag_unshard(parts, 2), x)
+        c = 12 // (2 * world)
+        assert torch.equal(parts[0][0][:c], x[:c])                     # rank 0 half 0: chunk 0 of sequence 0
+        assert torch.equal(parts[0][1][:c], x[12 - c:12])              # rank 0 half 1: the last chunk
